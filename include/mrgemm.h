@@ -1,0 +1,182 @@
+/*
+ * mrgemm.h -- C ABI of the weight-streaming multi-row matmul library
+ * (libmrgemm.so, sm_100a / B200).
+ *
+ * The library computes C[m,n] = A[m,k] . W[k,n] with the weight read from HBM
+ * once per call and shared by every row (the question the nx_batchscale_kat.nx
+ * note asks of a matmul path), the multi-row router GEMV and top-10 of Strata
+ * PR #109 ("What", router bullet), and the tiled f16/bf16 GEMM for prompt
+ * chunks of the "opus r35 track A" audit (section 2, gemm_f16 tiles).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.   Matrices are row-major with an explicit row stride in ELEMENTS.
+ *           The weight is passed k-contiguous as Wt[n][k]: row j of Wt is
+ *           column j of the logical W[k,n].  Logically C = A . W throughout.
+ * Memory.   Every pointer is a device pointer owned by the caller; the
+ *           library allocates no device memory per call.  Outputs are
+ *           written only by kernels, never by the host.
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *           default stream).  Calls are asynchronous on that stream and never
+ *           synchronise, except mr_poll_errors.
+ * Errors.   Arguments are validated on the host before any launch; on an
+ *           error nothing is launched and no output is touched.  No C++
+ *           exception crosses the ABI.  The entry points are re-entrant and
+ *           thread-safe.
+ * Device.   Every wait inside a kernel is bounded in time; a wait that runs
+ *           out records a bit in a per-device error word (read it with
+ *           mr_poll_errors) and the kernel returns without completing.
+ * Numerics. Inputs are exact 16-bit floats, products are accumulated in fp32
+ *           in a fixed order, and there is no split-K or stream-K: the bits of
+ *           an output element depend only on its row of A, its row of Wt and
+ *           k -- not on m, on the other rows, or on the tile shape chosen.
+ */
+#ifndef MRGEMM_H
+#define MRGEMM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mr_status {
+    MR_OK = 0,
+    MR_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, stride < row length */
+    MR_ERR_MISALIGNED = 2,    /* pointer not 16-byte aligned, or k / stride not a multiple of 8 */
+    MR_ERR_UNSUPPORTED = 3,   /* size beyond what this build handles (documented per call) */
+    MR_ERR_CUDA = 4,          /* a CUDA runtime call failed (no device, launch error, ...) */
+    MR_ERR_TIMEOUT = 5        /* a bounded device wait ran out (see mr_poll_errors) */
+} mr_status;
+
+/* Element types. */
+enum { MR_F16 = 0, MR_BF16 = 1, MR_F32 = 2 };
+
+/* Bits of the per-device error word returned by mr_poll_errors. */
+#define MR_DEVERR_GEMV_TIMEOUT   0x1u   /* mrgemv_bf16: a weight stage never arrived */
+#define MR_DEVERR_GEMM_TIMEOUT   0x2u   /* gemm_f16: a TMA / MMA pipeline wait ran out */
+#define MR_DEVERR_TOPK_TIMEOUT   0x4u   /* router_topk: a wait ran out */
+#define MR_DEVERR_SELFTEST       0x8u   /* mr_selftest_wait_timeout fired as intended */
+
+/* Flags for mrgemv_bf16_ex. */
+#define MR_GEMV_PDL 0x1u
+/*
+ * MR_GEMV_PDL: launch with programmatic dependent launch.  The kernel starts
+ * streaming its weight into shared memory BEFORE the previous kernel on the
+ * stream has finished, and waits for that kernel only before it reads A.
+ * Use it only when the weight is not written by the kernel just before on the
+ * same stream (static weights are the normal case); A and C keep ordinary
+ * stream order.  Outputs are bitwise identical with and without the flag.
+ */
+
+/*
+ * mrgemv_bf16 -- multi-row bf16 GEMV, fp32 output.
+ *
+ * The multi-row GEMV of Strata PR #109 ("What", router bullet: one multi-row
+ * GEMV that reads the weight once with per-token accumulators in exactly the
+ * single-row order) and the "m>1 packed path" of the nx_batchscale_kat.nx note.
+ *
+ *   C[i][j] = sum_p A[i][p] * Wt[j][p]   for i < m, j < n, p < k
+ *
+ * A  : m rows of k bf16, row stride lda (>= k) elements, device.
+ * Wt : n rows of k bf16, row stride ldw (>= k) elements, device.
+ * C  : m rows of n fp32, row stride ldc (>= n) elements, device (written).
+ * 1 <= m <= 16 per call (larger m: call in groups of rows, each row's bits
+ * are unchanged); n >= 1; 8 <= k, k % 8 == 0; lda, ldw % 8 == 0; A and Wt
+ * 16-byte aligned; k no larger than the per-CTA shared memory allows
+ * (k <= 4096 is always accepted) -- else MR_ERR_UNSUPPORTED.
+ * Every weight byte is read from HBM once per call.  Row i's result is
+ * bitwise identical for every m and every position of the row in A.
+ */
+mr_status mrgemv_bf16(const void *A, int64_t lda, const void *Wt, int64_t ldw,
+                      float *C, int64_t ldc, int32_t m, int32_t n, int32_t k,
+                      void *stream);
+
+/* As mrgemv_bf16, with MR_GEMV_* flags (0 gives exactly mrgemv_bf16). */
+mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw,
+                         float *C, int64_t ldc, int32_t m, int32_t n, int32_t k,
+                         uint32_t flags, void *stream);
+
+/*
+ * router_topk -- per-row top-k of fp32 logits, one CTA per row.
+ *
+ * The multi-row top-10 launch of Strata PR #109 ("What", router bullet: the
+ * kernel takes blockIdx.x = token).  Order: value descending; equal values
+ * (-0.0 equals +0.0) by index ascending; a NaN ranks above +inf.  The result
+ * is unique under this total order.
+ *
+ * logits : m rows of n fp32, row stride ldl (>= n) elements, device.
+ * idx    : m rows of topk int32 (row stride ldo >= topk), written in rank order.
+ * val    : NULL, or m rows of topk fp32 (row stride ldo): the logits at idx,
+ *          bit for bit.
+ * 1 <= m <= 2^31-1; 1 <= n; 1 <= topk <= min(n, 32).
+ */
+mr_status router_topk(const float *logits, int64_t ldl, int32_t m, int32_t n,
+                      int32_t topk, int32_t *idx, float *val, int64_t ldo,
+                      void *stream);
+
+/*
+ * gemm_f16 -- tiled GEMM on the tcgen05 tensor cores (TMA -> shared memory
+ * -> tcgen05.mma with the accumulator in tensor memory), fp32 accumulate.
+ *
+ * The gemm_f16<TM,TN,SG> prompt-chunk GEMM of the "opus r35 track A" audit
+ * (section 2: tiles for M = 150..2048, the M % 128 tail-tile rule, bitwise
+ * parity across tiles), rebuilt for sm_100a.
+ *
+ *   C[i][j] = sum_p A[i][p] * Wt[j][p]     (fp32 accumulate, then out_dtype)
+ *
+ * A  : M rows of K elements of in_dtype (MR_F16 or MR_BF16), stride lda.
+ * Wt : N rows of K elements of in_dtype, stride ldw.
+ * C  : M rows of N elements of out_dtype (MR_F16, MR_BF16 or MR_F32), stride ldc;
+ *      16-bit outputs are rounded to nearest even.
+ * tile_id : -1 selects with gemm_f16_select_tile; 0 .. gemm_f16_num_tiles()-1
+ *      forces a tile.  Every tile gives the same bits (fixed K order, K steps of
+ *      16, no split-K).
+ * M, N >= 1; K >= 8, K % 8 == 0; lda, ldw, ldc % 8 == 0; A, Wt, C 16-byte aligned.
+ */
+mr_status gemm_f16(const void *A, int64_t lda, const void *Wt, int64_t ldw,
+                   void *C, int64_t ldc, int32_t M, int32_t N, int32_t K,
+                   int32_t in_dtype, int32_t out_dtype, int32_t tile_id,
+                   void *stream);
+
+/* Number of tile shapes gemm_f16 can run. */
+int32_t gemm_f16_num_tiles(void);
+
+/* "BMxBN" name of a tile id (e.g. "128x96"), or NULL when out of range. */
+const char *gemm_f16_tile_name(int32_t tile_id);
+
+/*
+ * The tile gemm_f16 picks for (M, N, K) when tile_id is -1: a host-side
+ * integer cost model over the machine's SM count -- padded tail tiles
+ * (M % 128 in 1..64 wastes up to half a tile), wave quantisation, and the
+ * narrow-N case (N = 96).  Returns -1 for invalid sizes.
+ */
+int32_t gemm_f16_select_tile(int32_t M, int32_t N, int32_t K);
+
+/*
+ * mr_poll_errors -- synchronise `stream`, then read and clear the error word
+ * of the current device.  *device_flags receives MR_DEVERR_* bits (0 when all
+ * waits completed).  Returns MR_ERR_TIMEOUT if any bit was set, MR_ERR_CUDA if
+ * the synchronisation failed, else MR_OK.  device_flags may be NULL.
+ */
+mr_status mr_poll_errors(void *stream, uint32_t *device_flags);
+
+/*
+ * mr_selftest_wait_timeout -- launch one CTA that waits on an mbarrier which
+ * nothing will ever complete, bounded by limit_us microseconds (1..1000000).
+ * The wait runs out, sets MR_DEVERR_SELFTEST, and the kernel returns
+ * normally: it exercises the bounded-wait path without faulting the GPU.
+ */
+mr_status mr_selftest_wait_timeout(int32_t limit_us, void *stream);
+
+/* Human-readable name of a status code. */
+const char *mr_status_str(mr_status status);
+
+/* Library version string. */
+const char *mr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MRGEMM_H */

@@ -1,0 +1,81 @@
+"""The C ABI on a machine without a GPU: exports, validation, status codes.
+
+Only host-side validation runs here; every call below returns before any CUDA
+call is made, except the one that checks a valid call reports MR_ERR_CUDA
+when no device exists.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import verify_weight_streaming_b200 as mr
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "mrgemm.h")
+P = ctypes.c_void_p
+A16 = P(256)            # 16-byte aligned stand-in pointers (never dereferenced)
+BAD = P(258)            # 2-byte aligned
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_0-9]+)\s*\(", text)) - {"defined"})
+
+
+def test_header_declares_and_library_exports_every_entry_point():
+    names = declared_functions()
+    assert set(mr.EXPORTS) <= set(names), set(mr.EXPORTS) - set(names)
+    for name in names:
+        assert hasattr(mr.lib, name), f"libmrgemm.so does not export {name}"
+
+
+def test_status_strings():
+    for code, name in enumerate(["MR_OK", "MR_ERR_INVALID_ARG", "MR_ERR_MISALIGNED",
+                                 "MR_ERR_UNSUPPORTED", "MR_ERR_CUDA", "MR_ERR_TIMEOUT"]):
+        assert mr.status_str(code) == name
+    assert mr.status_str(99) == "MR_ERR_UNKNOWN"
+    assert "sm_100a" in mr.version()
+
+
+def gemv(A=A16, lda=64, W=A16, ldw=64, C=A16, ldc=32, m=4, n=32, k=64, flags=0):
+    return mr.lib.mrgemv_bf16_ex(A, lda, W, ldw, C, ldc, m, n, k, flags, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(A=None), mr.MR_ERR_INVALID_ARG), (dict(W=None), mr.MR_ERR_INVALID_ARG),
+    (dict(C=None), mr.MR_ERR_INVALID_ARG), (dict(m=0), mr.MR_ERR_INVALID_ARG),
+    (dict(n=0), mr.MR_ERR_INVALID_ARG), (dict(k=0), mr.MR_ERR_INVALID_ARG),
+    (dict(lda=56), mr.MR_ERR_INVALID_ARG), (dict(ldc=31), mr.MR_ERR_INVALID_ARG),
+    (dict(flags=2), mr.MR_ERR_INVALID_ARG),
+    (dict(k=60, lda=64, ldw=64), mr.MR_ERR_MISALIGNED), (dict(lda=68), mr.MR_ERR_MISALIGNED),
+    (dict(A=BAD), mr.MR_ERR_MISALIGNED), (dict(W=BAD), mr.MR_ERR_MISALIGNED),
+    (dict(m=17), mr.MR_ERR_UNSUPPORTED),
+])
+def test_gemv_validation(kw, code):
+    assert gemv(**kw) == code
+
+
+def test_gemv_valid_call_without_device_is_a_cuda_error():
+    assert gemv() == mr.MR_ERR_CUDA
+
+
+def topk(logits=A16, ldl=512, m=4, n=512, k=10, idx=A16, val=None, ldo=10):
+    return mr.lib.router_topk(logits, ldl, m, n, k, idx, val, ldo, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(logits=None), mr.MR_ERR_INVALID_ARG), (dict(idx=None), mr.MR_ERR_INVALID_ARG),
+    (dict(m=0), mr.MR_ERR_INVALID_ARG), (dict(n=0), mr.MR_ERR_INVALID_ARG),
+    (dict(k=0), mr.MR_ERR_INVALID_ARG), (dict(n=8, ldl=8, k=9, ldo=9), mr.MR_ERR_INVALID_ARG),
+    (dict(ldl=500), mr.MR_ERR_INVALID_ARG), (dict(ldo=9), mr.MR_ERR_INVALID_ARG),
+    (dict(k=33, ldo=33), mr.MR_ERR_UNSUPPORTED), (dict(logits=P(258)), mr.MR_ERR_MISALIGNED),
+])
+def test_topk_validation(kw, code):
+    assert topk(**kw) == code
+
+
+def test_selftest_limits():
+    assert mr.lib.mr_selftest_wait_timeout(0, None) == mr.MR_ERR_INVALID_ARG
+    assert mr.lib.mr_selftest_wait_timeout(1000001, None) == mr.MR_ERR_INVALID_ARG

@@ -1,0 +1,142 @@
+"""mrgemv_bf16 on the GPU against the fp64 oracle, plus bitwise batch invariance.
+
+Pass bar (per element): |C_gpu - C64| <= 1e-5 * sum|a*w|.  Bitwise: row i of
+the output is the same for every m in 1..16 and every position in A, with and
+without programmatic dependent launch.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import dev_bits, host, need_gpu, padded, torch
+
+import verify_weight_streaming_b200 as mr
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+    yield
+    assert mr.mr_poll_errors() == 0
+
+
+def run_gemv(a_bits, w_bits, flags=0, ldc=None, lda=None, ldw=None):
+    m, k = a_bits.shape
+    n = w_bits.shape[0]
+    A = dev_bits(a_bits)
+    if lda is not None:
+        buf, A2 = padded(m, k, lda, torch.int16, 0x7FC0)
+        A2.copy_(A)
+        A = A2
+    W = dev_bits(w_bits)
+    if ldw is not None:
+        buf, W2 = padded(n, k, ldw, torch.int16, 0x7FC0)
+        W2.copy_(W)
+        W = W2
+    ldc = ldc or n
+    cbuf = torch.full((m + 1, ldc), float("nan"), dtype=torch.float32, device="cuda")
+    C = cbuf[:m, :n]
+    mr.mrgemv_bf16(A, W, C, flags=flags)
+    out = host(cbuf)
+    # canaries: padding columns and the spare row are untouched
+    assert np.isnan(out[:m, n:]).all() and np.isnan(out[m]).all()
+    return out[:m, :n]
+
+
+def check(c, a_bits, w_bits):
+    c64, s64 = oracle.matmul(a_bits, "bf16", w_bits, "bf16")
+    ok, worst, where = oracle.check_matmul(c, c64, s64)
+    assert ok, f"worst |err|/tol = {worst:.3g} at {where}"
+    return worst
+
+
+@pytest.mark.parametrize("m", [1, 2, 4, 8, 16])
+def test_ffn_shape_parity(m):
+    """A[m,896] x W[896,4864] (the KAT's Qwen FFN inner dim)."""
+    a, w = synth.gemv_ffn(m)
+    check(run_gemv(a, w), a, w)
+
+
+@pytest.mark.parametrize("m", [1, 2, 4, 8, 16])
+def test_router_shape_parity(m):
+    """A[m,2560] x W_r[2560,512] (the 2.6 MB router)."""
+    a, w = synth.router(m)
+    check(run_gemv(a, w), a, w)
+
+
+def test_sweep_shape_parity_ring_refill():
+    """K=2560, N=6144: more column groups than ring slots, so slots are refilled."""
+    a = synth.normal_bits(synth.seed_for(synth.WL_SWEEP, 0), (16, 2560), "bf16", 1.0)
+    w = synth.normal_bits(synth.seed_for(synth.WL_SWEEP, 1), (6144, 2560), "bf16", 1.0 / np.sqrt(2560))
+    check(run_gemv(a, w), a, w)
+
+
+@pytest.mark.parametrize("m,n,k", [
+    (1, 1, 8), (3, 5, 24), (5, 33, 136), (16, 147, 1024), (7, 149, 2048), (2, 300, 520),
+    (16, 1000, 4096), (9, 2, 8), (11, 7, 4088),
+])
+def test_ragged_shapes(m, n, k):
+    a = synth.normal_bits(100 + k, (m, k), "bf16", 1.0)
+    w = synth.normal_bits(200 + n, (n, k), "bf16", 1.0 / np.sqrt(k))
+    check(run_gemv(a, w), a, w)
+
+
+def test_strided_operands_and_canaries():
+    a, w = synth.gemv_ffn(6, k=896, n=1000)
+    c = run_gemv(a, w, ldc=1016, lda=904, ldw=912)
+    check(c, a, w)
+
+
+def test_integer_inputs_are_exact():
+    """Small integers: every partial sum is an integer below 2^24, so fp32 is exact."""
+    for (m, n, k) in [(16, 300, 896), (4, 64, 2560)]:
+        a = synth.integer_bits(5, (m, k), "bf16", -15, 15)
+        w = synth.integer_bits(6, (n, k), "bf16", -15, 15)
+        c = run_gemv(a, w)
+        c64, _ = oracle.matmul(a, "bf16", w, "bf16")
+        assert np.array_equal(c.astype(np.float64), c64)
+
+
+@pytest.mark.parametrize("shape", ["ffn", "router", "ragged"])
+def test_rows_bitwise_identical_across_m(shape):
+    if shape == "ffn":
+        a, w = synth.gemv_ffn(16)
+    elif shape == "router":
+        a, w = synth.router(16)
+    else:
+        a = synth.normal_bits(9, (16, 1032), "bf16", 1.0)
+        w = synth.normal_bits(10, (77, 1032), "bf16", 0.03)
+    full = run_gemv(a, w)
+    for m in range(1, 16):
+        part = run_gemv(a[:m], w)
+        assert np.array_equal(part.view(np.uint32), full[:m].view(np.uint32)), f"m={m}"
+    # a row placed anywhere in the window gives the same bits
+    perm = np.random.default_rng(0).permutation(16)
+    pc = run_gemv(a[perm], w)
+    assert np.array_equal(pc.view(np.uint32), full[perm].view(np.uint32))
+    for i in (0, 5, 15):
+        single = run_gemv(a[i:i + 1], w)
+        assert np.array_equal(single.view(np.uint32), full[i:i + 1].view(np.uint32))
+
+
+def test_pdl_flag_gives_identical_bits():
+    a, w = synth.router(8)
+    plain = run_gemv(a, w)
+    pdl = run_gemv(a, w, flags=mr.MR_GEMV_PDL)
+    assert np.array_equal(plain.view(np.uint32), pdl.view(np.uint32))
+    a, w = synth.gemv_ffn(16)
+    assert np.array_equal(run_gemv(a, w).view(np.uint32),
+                          run_gemv(a, w, flags=mr.MR_GEMV_PDL).view(np.uint32))
+
+
+def test_bounded_wait_selftest_reports_and_context_survives():
+    assert mr.mr_poll_errors() == 0
+    mr.mr_selftest_wait_timeout(2000)
+    flags = mr.mr_poll_errors()
+    assert flags == mr.MR_DEVERR_SELFTEST
+    assert mr.mr_poll_errors() == 0
+    a, w = synth.router(2)
+    check(run_gemv(a, w), a, w)

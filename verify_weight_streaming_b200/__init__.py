@@ -1,0 +1,161 @@
+"""Python binding of libmrgemm.so (ctypes; argument marshalling only).
+
+Every function has the name of the C entry point it calls (see
+``include/mrgemm.h``).  Tensors are torch CUDA tensors: torch supplies device
+memory and the current stream, the library does all of the arithmetic.  16-bit
+inputs may be ``torch.bfloat16`` / ``torch.float16`` or raw ``torch.int16``
+patterns.  A status other than MR_OK raises ``MrError``.  If the compiled
+library is missing the import fails: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from ._build import LIB, build  # noqa: F401
+
+MR_OK, MR_ERR_INVALID_ARG, MR_ERR_MISALIGNED, MR_ERR_UNSUPPORTED, MR_ERR_CUDA, MR_ERR_TIMEOUT = range(6)
+MR_F16, MR_BF16, MR_F32 = 0, 1, 2
+MR_GEMV_PDL = 0x1
+MR_DEVERR_GEMV_TIMEOUT, MR_DEVERR_GEMM_TIMEOUT, MR_DEVERR_TOPK_TIMEOUT, MR_DEVERR_SELFTEST = 1, 2, 4, 8
+
+EXPORTS = (
+    "mrgemv_bf16", "mrgemv_bf16_ex", "router_topk", "gemm_f16", "gemm_f16_num_tiles",
+    "gemm_f16_tile_name", "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout",
+    "mr_status_str", "mr_version",
+)
+
+
+class MrError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call}: {status_str(status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB):
+        raise ImportError(f"{LIB} is not built; run __graft_entry__.build() (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB)
+    P, I64, I32, U32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32
+    L.mrgemv_bf16.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, P]
+    L.mrgemv_bf16_ex.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, U32, P]
+    L.router_topk.argtypes = [P, I64, I32, I32, I32, P, P, I64, P]
+    L.gemm_f16.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, I32, I32, P]
+    L.gemm_f16_num_tiles.argtypes = []
+    L.gemm_f16_tile_name.argtypes = [I32]
+    L.gemm_f16_tile_name.restype = ctypes.c_char_p
+    L.gemm_f16_select_tile.argtypes = [I32, I32, I32]
+    L.mr_poll_errors.argtypes = [P, ctypes.POINTER(U32)]
+    L.mr_selftest_wait_timeout.argtypes = [I32, P]
+    L.mr_status_str.argtypes = [ctypes.c_int]
+    L.mr_status_str.restype = ctypes.c_char_p
+    L.mr_version.argtypes = []
+    L.mr_version.restype = ctypes.c_char_p
+    for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "router_topk", "gemm_f16", "gemm_f16_num_tiles",
+                 "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout"):
+        getattr(L, name).restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.mr_status_str(int(status)).decode()
+
+
+def version() -> str:
+    return lib.mr_version().decode()
+
+
+def _check(status: int, call: str) -> None:
+    if status != MR_OK:
+        raise MrError(status, call)
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _rows(t, name):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D tensor with unit column stride")
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return {torch.float16: MR_F16, torch.bfloat16: MR_BF16, torch.float32: MR_F32,
+            torch.int16: MR_BF16}.get(t.dtype, -1)
+
+
+def mrgemv_bf16(A, Wt, C, stream=None, flags: int = 0) -> None:
+    """C[m,n] (fp32) = A[m,k] (bf16) . Wt[n,k]^T (bf16); m <= 16."""
+    m, k, lda = _rows(A, "A")
+    n, kw, ldw = _rows(Wt, "Wt")
+    mc, nc, ldc = _rows(C, "C")
+    if kw != k or mc != m or nc != n:
+        raise ValueError(f"shape mismatch A{tuple(A.shape)} Wt{tuple(Wt.shape)} C{tuple(C.shape)}")
+    st = lib.mrgemv_bf16_ex(A.data_ptr(), lda, Wt.data_ptr(), ldw, C.data_ptr(), ldc,
+                            m, n, k, flags, _stream(stream))
+    _check(st, "mrgemv_bf16")
+
+
+def router_topk(logits, topk: int, idx, val=None, stream=None) -> None:
+    """idx[m,topk] (int32), val[m,topk] (fp32, optional) = per-row top-k of logits[m,n]."""
+    m, n, ldl = _rows(logits, "logits")
+    mi, ki, ldo = _rows(idx, "idx")
+    if mi != m or ki < topk:
+        raise ValueError("idx shape mismatch")
+    vptr = None
+    if val is not None:
+        mv, kv, ldv = _rows(val, "val")
+        if mv != m or kv < topk or ldv != ldo:
+            raise ValueError("val must match idx's shape and stride")
+        vptr = val.data_ptr()
+    st = lib.router_topk(logits.data_ptr(), ldl, m, n, topk, idx.data_ptr(), vptr, ldo, _stream(stream))
+    _check(st, "router_topk")
+
+
+def gemm_f16(A, Wt, C, tile_id: int = -1, in_dtype: int | None = None, stream=None) -> None:
+    """C[M,N] = A[M,K] . Wt[N,K]^T on tcgen05; dtypes from the tensors (int16 = bf16 bits)."""
+    M, K, lda = _rows(A, "A")
+    N, kw, ldw = _rows(Wt, "Wt")
+    mc, nc, ldc = _rows(C, "C")
+    if kw != K or mc != M or nc != N:
+        raise ValueError("shape mismatch")
+    idt = _dtype_code(A) if in_dtype is None else in_dtype
+    st = lib.gemm_f16(A.data_ptr(), lda, Wt.data_ptr(), ldw, C.data_ptr(), ldc, M, N, K,
+                      idt, _dtype_code(C), tile_id, _stream(stream))
+    _check(st, "gemm_f16")
+
+
+def gemm_f16_num_tiles() -> int:
+    return int(lib.gemm_f16_num_tiles())
+
+
+def gemm_f16_tile_name(tile_id: int):
+    r = lib.gemm_f16_tile_name(tile_id)
+    return None if r is None else r.decode()
+
+
+def gemm_f16_select_tile(M: int, N: int, K: int) -> int:
+    return int(lib.gemm_f16_select_tile(M, N, K))
+
+
+def mr_poll_errors(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error bits."""
+    flags = ctypes.c_uint32(0)
+    st = lib.mr_poll_errors(_stream(stream), ctypes.byref(flags))
+    if st not in (MR_OK, MR_ERR_TIMEOUT):
+        raise MrError(st, "mr_poll_errors")
+    return int(flags.value)
+
+
+def mr_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    _check(lib.mr_selftest_wait_timeout(limit_us, _stream(stream)), "mr_selftest_wait_timeout")

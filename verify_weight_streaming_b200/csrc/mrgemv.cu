@@ -1,0 +1,436 @@
+// mrgemv_bf16: multi-row bf16 GEMV with fp32 output for m <= 16 rows.
+//
+// The multi-row GEMV of Strata PR #109 ("What", router bullet): the weight is
+// read from HBM once per call and shared by all m rows, and every row's
+// accumulators follow exactly the order of the single-row call.  The
+// nx_batchscale_kat.nx note states the test this has to pass: per-row cost must
+// fall with m because the weight bytes are not re-streamed per row.
+//
+// Design (B200):
+//  * grid = one CTA per SM (at most n); CTA b owns the contiguous column block
+//    [b*n/G, (b+1)*n/G) of Wt, i.e. a contiguous run of weight rows.
+//  * The block streams through a ring of shared-memory slots, one column group
+//    (up to CG columns x k) per slot, with cp.async.bulk global->shared copies
+//    counted on an mbarrier (no tensor map, no multicast).  The first slots are
+//    requested before griddepcontrol.wait, so under programmatic dependent
+//    launch the weight stream overlaps the previous kernel.
+//  * A (m rows, bf16) is staged once in shared memory; rows m..MB-1 are zero.
+//  * Lanes split k in 4-element chunks: chunk q belongs to lane q % 32 of the
+//    k-slice that holds it.  KW warps split k into contiguous slices; KW is a
+//    function of k alone.  Each lane keeps, per (row, column), two fp32
+//    accumulators (even / odd element of each pair) updated with
+//    fma.rn.f32x2 in ascending chunk order.
+//  * Reduction: even + odd, then a fixed xor-butterfly over the 32 lanes
+//    (bit 16, 8, 4, 2, 1; realised as a reduce-scatter so each lane finishes a
+//    share of the values), then the KW slices in slice order.  The tree of
+//    every output element is the same for every m, every row position and
+//    every column grouping, so row i is bitwise identical at every m.
+//  * Every wait is an mbarrier wait bounded in time; nothing uses bar.sync
+//    after the prologue, so a wait that runs out cannot strand other warps.
+#include "common.cuh"
+
+#include <algorithm>
+#include <mutex>
+
+namespace mr {
+namespace gemv {
+
+constexpr int kMaxWarps = 8;
+constexpr int kMaxRows = 16;
+
+struct Params {
+    const uint16_t *A;
+    int64_t lda;
+    const uint16_t *Wt;
+    int64_t ldw;
+    float *C;
+    int64_t ldc;
+    int m, n, k;
+    int G;          // CTAs
+    int KW;         // warps splitting k (function of k only)
+    int CWG;        // column-group warps per CTA
+    int S;          // ring slots
+    uint32_t a_bytes;     // shared bytes reserved for A (MB rows)
+    uint32_t slot_bytes;  // CG * k * 2
+};
+
+// k-slice split: a function of k alone (never of m), so the reduction tree of
+// an output element is fixed by k.
+__host__ __device__ inline int k_warps(int k) {
+    const int q = k / 4;
+    if (q % 128 == 0 && q >= 512) return 4;
+    if (q % 64 == 0 && q >= 256) return 2;
+    return 1;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// acc.x = fma(a.x, b.x, acc.x); acc.y = fma(a.y, b.y, acc.y), both round-to-nearest.
+__device__ __forceinline__ void ffma2(float2 &acc, float ax, float ay, float bx, float by) {
+    asm("{\n\t.reg .b64 a2, b2, c2;\n\t"
+        "mov.b64 a2, {%2, %3};\n\t"
+        "mov.b64 b2, {%4, %5};\n\t"
+        "mov.b64 c2, {%0, %1};\n\t"
+        "fma.rn.f32x2 c2, a2, b2, c2;\n\t"
+        "mov.b64 {%0, %1}, c2;\n\t}"
+        : "+f"(acc.x), "+f"(acc.y)
+        : "f"(ax), "f"(ay), "f"(bx), "f"(by));
+}
+
+// Reduce-scatter over the warp: level D pairs lanes that differ in bit D (16,
+// 8, 4, 2, 1 in that order).  While more than one value is left, the lane with
+// bit D clear keeps the lower half and its partner the upper half; with one
+// value left both partners add (a + b == b + a, so both hold the same bits).
+template <int CNT, int D>
+struct ReduceScatter {
+    static __device__ __forceinline__ void run(float *v, int lane, int &base) {
+        if constexpr (CNT >= 2) {
+            constexpr int H = CNT / 2;
+            const bool up = (lane & D) != 0;
+#pragma unroll
+            for (int i = 0; i < H; ++i) {
+                const float send = up ? v[i] : v[i + H];
+                const float keep = up ? v[i + H] : v[i];
+                const float recv = __shfl_xor_sync(0xffffffffu, send, D);
+                v[i] = __fadd_rn(keep, recv);
+            }
+            if (up) base += H;
+            if constexpr (D > 1) ReduceScatter<H, D / 2>::run(v, lane, base);
+        } else {
+            v[0] = __fadd_rn(v[0], __shfl_xor_sync(0xffffffffu, v[0], D));
+            if constexpr (D > 1) ReduceScatter<1, D / 2>::run(v, lane, base);
+        }
+    }
+};
+
+// Values per lane after the reduce-scatter of V values, and the mask of lane
+// bits that were butterfly (replicating) levels.
+template <int V>
+struct Scatter {
+    static constexpr int kPerLane = V >= 32 ? V / 32 : 1;
+    static constexpr int kReplMask = V >= 32 ? 0 : (32 / V) - 1;
+};
+
+struct Smem {
+    uint16_t *a;          // [MB][k]
+    uint8_t *ring;        // S slots
+    uint64_t *full;       // [S]
+    uint64_t *empty;      // [S]
+    uint64_t *red_full;   // [CWG]
+    uint64_t *red_free;   // [CWG]
+    float *red;           // [CWG][KW][32][VPL]
+};
+
+// One column group: NC (power of two) columns of this warp's k-slice.
+template <int MB, int NC, int VPL>
+__device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g, int ncol,
+                                         int col0, int slice, int cw, int it, int lane,
+                                         int q_begin, int q_end) {
+    const int k = p.k;
+    const int slot = g % p.S;
+    const uint32_t par = (uint32_t)(g / p.S) & 1u;
+    if (!mbar_wait_bounded(smem_u32(&sm.full[slot]), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
+
+    const uint16_t *w = reinterpret_cast<const uint16_t *>(sm.ring + (size_t)slot * p.slot_bytes);
+    float2 acc[MB][NC];
+#pragma unroll
+    for (int r = 0; r < MB; ++r)
+#pragma unroll
+        for (int j = 0; j < NC; ++j) acc[r][j] = make_float2(0.f, 0.f);
+
+#pragma unroll 2
+    for (int q = q_begin + lane; q < q_end; q += 32) {
+        float w0[NC], w1[NC], w2[NC], w3[NC];
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+            const uint2 raw = *reinterpret_cast<const uint2 *>(w + (size_t)j * k + 4 * q);
+            w0[j] = bf16lo(raw.x);
+            w1[j] = bf16hi(raw.x);
+            w2[j] = bf16lo(raw.y);
+            w3[j] = bf16hi(raw.y);
+        }
+#pragma unroll
+        for (int r = 0; r < MB; ++r) {
+            const uint2 ar = *reinterpret_cast<const uint2 *>(sm.a + (size_t)r * k + 4 * q);
+            const float a0 = bf16lo(ar.x), a1 = bf16hi(ar.x);
+            const float a2 = bf16lo(ar.y), a3 = bf16hi(ar.y);
+#pragma unroll
+            for (int j = 0; j < NC; ++j) {
+                ffma2(acc[r][j], a0, a1, w0[j], w1[j]);
+                ffma2(acc[r][j], a2, a3, w2[j], w3[j]);
+            }
+        }
+    }
+    // This warp no longer reads the slot.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&sm.empty[slot]));
+
+    constexpr int V = MB * NC;
+    float v[V];
+#pragma unroll
+    for (int r = 0; r < MB; ++r)
+#pragma unroll
+        for (int j = 0; j < NC; ++j) v[r * NC + j] = __fadd_rn(acc[r][j].x, acc[r][j].y);
+    int base = 0;
+    ReduceScatter<V, 16>::run(v, lane, base);
+    constexpr int PL = Scatter<V>::kPerLane;
+
+    bool ok = true;
+    if (p.KW > 1) {
+        float *red = sm.red + (size_t)cw * p.KW * 32 * VPL;
+        const uint32_t rpar = (uint32_t)it & 1u;
+        if (slice > 0) {
+            // Wait until slice 0 has consumed the previous group's partials.
+            if (it > 0)
+                ok = mbar_wait_bounded(smem_u32(&sm.red_free[cw]), rpar ^ 1u, MR_DEVERR_GEMV_TIMEOUT);
+            if (ok) {
+#pragma unroll
+                for (int i = 0; i < PL; ++i) red[((size_t)slice * 32 + lane) * VPL + i] = v[i];
+                mbar_arrive(smem_u32(&sm.red_full[cw]));
+            }
+        } else {
+            ok = mbar_wait_bounded(smem_u32(&sm.red_full[cw]), rpar, MR_DEVERR_GEMV_TIMEOUT);
+            if (ok) {
+                for (int s = 1; s < p.KW; ++s)
+#pragma unroll
+                    for (int i = 0; i < PL; ++i)
+                        v[i] = __fadd_rn(v[i], red[((size_t)s * 32 + lane) * VPL + i]);
+                mbar_arrive(smem_u32(&sm.red_free[cw]));
+            }
+        }
+    }
+
+    if (ok && slice == 0 && (lane & Scatter<V>::kReplMask) == 0) {
+#pragma unroll
+        for (int i = 0; i < PL; ++i) {
+            const int idx = base + i;
+            const int r = idx / NC, j = idx % NC;
+            if (r < p.m && j < ncol) p.C[(int64_t)r * p.ldc + col0 + j] = v[i];
+        }
+    }
+    return ok;
+}
+
+// Run a group of `ncol` valid columns with the smallest power-of-two width
+// NC >= ncol (extra columns compute on whatever the slot holds and are never
+// stored; every column's arithmetic is independent of NC).
+template <int MB, int NC, int VPL>
+__device__ __forceinline__ bool run_group(const Params &p, const Smem &sm, int g, int ncol,
+                                          int col0, int slice, int cw, int it, int lane,
+                                          int q_begin, int q_end) {
+    if constexpr (NC > 1) {
+        if (ncol <= NC / 2)
+            return run_group<MB, NC / 2, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end);
+    }
+    return do_group<MB, NC, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end);
+}
+
+template <int MB, int CG>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    constexpr int VPL = Scatter<MB * CG>::kPerLane;
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int k = p.k;
+
+    // Column block of this CTA.
+    const int c_begin = (int)(((int64_t)blockIdx.x * p.n) / p.G);
+    const int c_end = (int)(((int64_t)(blockIdx.x + 1) * p.n) / p.G);
+    const int ncols = c_end - c_begin;
+    const int ng = (ncols + CG - 1) / CG;
+
+    Smem sm;
+    sm.a = reinterpret_cast<uint16_t *>(smem_raw);
+    sm.ring = smem_raw + p.a_bytes;
+    sm.full = reinterpret_cast<uint64_t *>(sm.ring + (size_t)p.S * p.slot_bytes);
+    sm.empty = sm.full + p.S;
+    sm.red_full = sm.empty + p.S;
+    sm.red_free = sm.red_full + p.CWG;
+    sm.red = reinterpret_cast<float *>(sm.red_free + p.CWG);
+
+    auto issue_group = [&](int g) {
+        const int slot = g % p.S;
+        const int gc0 = c_begin + g * CG;
+        const int nc = min(CG, c_end - gc0);
+        const uint32_t row_bytes = (uint32_t)k * 2u;
+        const uint32_t bar = smem_u32(&sm.full[slot]);
+        const uint32_t dst = smem_u32(sm.ring + (size_t)slot * p.slot_bytes);
+        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)nc);
+        if (p.ldw == k) {
+            bulk_g2s(dst, p.Wt + (int64_t)gc0 * k, row_bytes * (uint32_t)nc, bar);
+        } else {
+            for (int j = 0; j < nc; ++j)
+                bulk_g2s(dst + j * row_bytes, p.Wt + (int64_t)(gc0 + j) * p.ldw, row_bytes, bar);
+        }
+    };
+
+    if (tid == 0) {
+        for (int s = 0; s < p.S; ++s) {
+            mbar_init(smem_u32(&sm.full[s]), 1);
+            mbar_init(smem_u32(&sm.empty[s]), (uint32_t)p.KW);
+        }
+        if (p.KW > 1) {
+            for (int c = 0; c < p.CWG; ++c) {
+                mbar_init(smem_u32(&sm.red_full[c]), (uint32_t)(p.KW - 1) * 32u);
+                mbar_init(smem_u32(&sm.red_free[c]), 32u);
+            }
+        }
+        fence_mbar_init();
+        const int first = min(ng, p.S);
+        for (int g = 0; g < first; ++g) issue_group(g);
+    }
+    // The weight stream is in flight; the next kernel may start launching.
+    grid_launch_dependents();
+    // A may be produced by the previous kernel on the stream.
+    grid_dependency_wait();
+
+    // Stage A (bf16) in shared memory; rows m..MB-1 are zero.
+    {
+        const int chunks = k / 8;  // 16-byte chunks per row
+        for (int e = tid; e < MB * chunks; e += blockDim.x) {
+            const int r = e / chunks, c = e % chunks;
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (r < p.m) val = *reinterpret_cast<const uint4 *>(p.A + (int64_t)r * p.lda + 8 * c);
+            *reinterpret_cast<uint4 *>(sm.a + (size_t)r * k + 8 * c) = val;
+        }
+    }
+    __syncthreads();
+
+    const int slice = warp % p.KW;
+    const int cw = warp / p.KW;
+    const int q_total = k / 4;
+    const int q_begin = (int)(((int64_t)slice * q_total) / p.KW);
+    const int q_end = (int)(((int64_t)(slice + 1) * q_total) / p.KW);
+
+    int it = 0;
+    for (int g = cw; g < ng; g += p.CWG, ++it) {
+        const int col0 = c_begin + g * CG;
+        const int ncol = min(CG, c_end - col0);
+        const bool ok = run_group<MB, CG, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end);
+        if (!ok) return;
+        // Refill the slot with group g + S once every slice has released it.
+        if (slice == 0 && lane == 0 && g + p.S < ng) {
+            const int slot = g % p.S;
+            const uint32_t par = (uint32_t)(g / p.S) & 1u;
+            if (!mbar_wait_bounded(smem_u32(&sm.empty[slot]), par, MR_DEVERR_GEMV_TIMEOUT)) return;
+            issue_group(g + p.S);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+using KernelFn = void (*)(const Params);
+
+template <int MB>
+constexpr int col_group() { return MB <= 8 ? 8 : 4; }
+
+KernelFn kernel_for(int MB) {
+    switch (MB) {
+        case 1: return gemv_kernel<1, col_group<1>()>;
+        case 2: return gemv_kernel<2, col_group<2>()>;
+        case 4: return gemv_kernel<4, col_group<4>()>;
+        case 8: return gemv_kernel<8, col_group<8>()>;
+        default: return gemv_kernel<16, col_group<16>()>;
+    }
+}
+
+int row_bucket(int m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
+
+std::mutex g_attr_mutex;
+bool g_attr_done[64] = {};
+
+cudaError_t ensure_attributes(int device) {
+    std::lock_guard<std::mutex> lock(g_attr_mutex);
+    if (device >= 0 && device < 64 && g_attr_done[device]) return cudaSuccess;
+    const int optin = mr_host::max_smem_optin();
+    const int mbs[] = {1, 2, 4, 8, 16};
+    for (int mb : mbs) {
+        cudaError_t e = cudaFuncSetAttribute(kernel_for(mb), cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        if (e != cudaSuccess) return e;
+    }
+    if (device >= 0 && device < 64) g_attr_done[device] = true;
+    return cudaSuccess;
+}
+
+}  // namespace gemv
+}  // namespace mr
+
+extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw,
+                                    float *C, int64_t ldc, int32_t m, int32_t n, int32_t k,
+                                    uint32_t flags, void *stream) {
+    using namespace mr::gemv;
+    if (!A || !Wt || !C) return MR_ERR_INVALID_ARG;
+    if (m < 1 || n < 1 || k < 1) return MR_ERR_INVALID_ARG;
+    if (lda < k || ldw < k || ldc < n) return MR_ERR_INVALID_ARG;
+    if (flags & ~MR_GEMV_PDL) return MR_ERR_INVALID_ARG;
+    if (k % 8 != 0 || lda % 8 != 0 || ldw % 8 != 0) return MR_ERR_MISALIGNED;
+    if (((uintptr_t)A & 15u) || ((uintptr_t)Wt & 15u) || ((uintptr_t)C & 3u)) return MR_ERR_MISALIGNED;
+    if (m > kMaxRows) return MR_ERR_UNSUPPORTED;
+
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) return mr_host::cuda_status(e);
+    const int sms = mr_host::sm_count();
+    const int optin = mr_host::max_smem_optin();
+    if (sms <= 0 || optin <= 0) return MR_ERR_CUDA;
+
+    Params p;
+    p.A = static_cast<const uint16_t *>(A);
+    p.lda = lda;
+    p.Wt = static_cast<const uint16_t *>(Wt);
+    p.ldw = ldw;
+    p.C = C;
+    p.ldc = ldc;
+    p.m = m;
+    p.n = n;
+    p.k = k;
+    const int MB = row_bucket(m);
+    const int CG = MB <= 8 ? 8 : 4;
+    p.KW = k_warps(k);
+    p.G = std::min(sms, n);
+    const int cols_max = (n + p.G - 1) / p.G;
+    const int ng_max = (cols_max + CG - 1) / CG;
+    p.CWG = std::max(1, std::min(ng_max, kMaxWarps / p.KW));
+    p.a_bytes = (uint32_t)(((size_t)MB * k * 2 + 127) / 128 * 128);
+    p.slot_bytes = (uint32_t)CG * (uint32_t)k * 2u;
+    const int vpl = std::max(1, MB * CG / 32);
+    const size_t fixed = p.a_bytes + 16 * (size_t)(2 * ng_max + 2 * p.CWG) +
+                         (size_t)p.CWG * p.KW * 32 * vpl * 4 + 64;
+    const size_t pdl_budget = 110 * 1024;
+    size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, optin) : (size_t)optin;
+    auto slots_for = [&](size_t b) -> int {
+        if (b <= fixed) return 0;
+        return (int)std::min<size_t>((size_t)ng_max, (b - fixed) / p.slot_bytes);
+    };
+    p.S = slots_for(budget);
+    if (p.S < 1) p.S = slots_for((size_t)optin);
+    if (p.S < 1) return MR_ERR_UNSUPPORTED;
+    const size_t smem = p.a_bytes + (size_t)p.S * p.slot_bytes + 16 * (size_t)(p.S + p.CWG) +
+                        (size_t)p.CWG * p.KW * 32 * vpl * 4;
+    if (smem > (size_t)optin) return MR_ERR_UNSUPPORTED;
+
+    e = ensure_attributes(device);
+    if (e != cudaSuccess) return mr_host::cuda_status(e);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.G);
+    cfg.blockDim = dim3((unsigned)(p.KW * p.CWG * 32));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (flags & MR_GEMV_PDL) ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kernel_for(MB), p);
+    return mr_host::cuda_status(e);
+}
+
+extern "C" mr_status mrgemv_bf16(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *C,
+                                 int64_t ldc, int32_t m, int32_t n, int32_t k, void *stream) {
+    return mrgemv_bf16_ex(A, lda, Wt, ldw, C, ldc, m, n, k, 0u, stream);
+}
