@@ -295,25 +295,6 @@ class RouterBench:
             graphs.append(g)
         return graphs
 
-    def capture_gemv_run(self, m, launches, flags):
-        torch, mr = self.torch, self.mr
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=self.stream):
-            for _ in range(launches):
-                mr.mrgemv_bf16(self.A[:m], self._next_w(), self.C[m], flags=flags)
-        return g
-
-    def capture_single_row_run(self, m, launches, flags):
-        """The per-row-launch mode: m separate m=1 calls per window (no batching)."""
-        torch, mr = self.torch, self.mr
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=self.stream):
-            for _ in range(launches):
-                w = self._next_w()
-                for r in range(m):
-                    mr.mrgemv_bf16(self.A[r:r + 1], w, self.C[m][r:r + 1], flags=flags)
-        return g
-
     def time_graphs(self, graphs, reps):
         torch = self.torch
         start = torch.cuda.Event(enable_timing=True)
@@ -368,18 +349,7 @@ def run_gpu(args, world, rank, local):
     clocks["sampled_over_us"] = elapsed_us + sum(extra)
 
     # ---- per-m curve and the GEMV roofline (back-to-back graph-captured calls)
-    curve = {}
-    launches = min(rb.pool, 64)
-    for m in WINDOWS:
-        g = [rb.capture_gemv_run(m, launches, flags) for _ in range(2)]
-        rb.time_graphs(g, 2)
-        t = min(rb.time_graphs(g, 8) / (8 * launches) for _ in range(3))
-        gs = [rb.capture_single_row_run(m, max(1, launches // m), flags)]
-        rb.time_graphs(gs, 1)
-        t1 = rb.time_graphs(gs, 4) / (4 * max(1, launches // m))
-        nbytes = gemv_bytes(m, N_ROUTER, K_ROUTER)
-        curve[str(m)] = {"us_per_call": t, "us_per_row": t / m, "GBps": nbytes / (t * 1e3),
-                         "per_row_launch_us_per_row": t1 / m}
+    curve = gemv_curve(rb, rb.W, rb.A, K_ROUTER, N_ROUTER, flags)
     speedup = curve["1"]["us_per_row"] / curve["8"]["us_per_row"]
     # dominant kernel: the GEMV, averaged over the step's mix of m
     mean_call_us = sum(curve[str(m)]["us_per_call"] for m in WINDOWS) / len(WINDOWS)
@@ -388,6 +358,9 @@ def run_gpu(args, world, rank, local):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": recorded_traffic("gemv_router"),
                 "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "mrgemv_bf16 (router, m mix 1..16)"}
+    extra_curves = {}
+    if not args.quick:
+        extra_curves = other_gemv_curves(rb, flags)
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(rb, args, world, device)
@@ -408,13 +381,81 @@ def run_gpu(args, world, rank, local):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(), "gpu_launches": args.steps * 2 * len(WINDOWS),
             "device_errors": errs, "clocks": clocks, "roofline": roofline,
-            "curve": {"router": curve, "batching_speedup_m1_over_m8": speedup},
+            "curve": {"router": curve, "batching_speedup_m1_over_m8": speedup, **extra_curves},
             "e2e": e2e, "gemm": gemm, "cpu_baseline": cpu,
             "pdl": not args.no_pdl,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def gemv_curve(rb, pool, A, k, n, flags, launches=None):
+    """us per call / per row and GB/s for each m, from graphs of back-to-back
+    calls over distinct weight copies; plus the per-row-launch mode (m calls
+    of m=1, the unbatched baseline)."""
+    torch, mr = rb.torch, rb.mr
+    launches = launches or min(len(pool), 64)
+    C = torch.empty((16, n), dtype=torch.float32, device=rb.device)
+    cursor = [0]
+
+    def nxt():
+        w = pool[cursor[0] % len(pool)]
+        cursor[0] += 1
+        return w
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=rb.stream):
+            fn()
+        return g
+
+    out = {}
+    for m in WINDOWS:
+        def batched():
+            for _ in range(launches):
+                mr.mrgemv_bf16(A[:m], nxt(), C[:m], flags=flags)
+
+        def per_row():
+            for _ in range(max(1, launches // m)):
+                w = nxt()
+                for r in range(m):
+                    mr.mrgemv_bf16(A[r:r + 1], w, C[r:r + 1], flags=flags)
+        with torch.cuda.stream(rb.stream):
+            batched()
+            per_row()
+        torch.cuda.synchronize()
+        g = [capture(batched) for _ in range(2)]
+        rb.time_graphs(g, 2)
+        t = min(rb.time_graphs(g, 8) / (8 * launches) for _ in range(3))
+        gs = [capture(per_row)]
+        rb.time_graphs(gs, 1)
+        t1 = min(rb.time_graphs(gs, 4) / (4 * max(1, launches // m)) for _ in range(2))
+        nbytes = gemv_bytes(m, n, k)
+        out[str(m)] = {"us_per_call": t, "us_per_row": t / m, "GBps": nbytes / (t * 1e3),
+                       "per_row_launch_us_per_row": t1 / m}
+    return out
+
+
+def other_gemv_curves(rb, flags):
+    """The KAT's FFN shape (k=896, n=4864) and the sweep shape (k=2560, n=6144)."""
+    import numpy as np
+    import synth
+    torch = rb.torch
+    res = {}
+    for name, k, n, wl in (("ffn_k896_n4864", 896, 4864, synth.WL_GEMV_FFN),
+                           ("sweep_k2560_n6144", 2560, 6144, synth.WL_SWEEP)):
+        a16 = synth.normal_bits(synth.seed_for(wl, 0), (16, k), "bf16", 1.0)
+        w16 = synth.normal_bits(synth.seed_for(wl, 1), (n, k), "bf16", 1.0 / np.sqrt(k))
+        w = torch.from_numpy(w16.view(np.int16)).to(rb.device)
+        copies = max(4, int(math.ceil(2.2 * rb.l2 / w16.nbytes)))
+        pool = [w.clone() for _ in range(copies)]
+        A = torch.from_numpy(a16.view(np.int16)).to(rb.device)
+        c = gemv_curve(rb, pool, A, k, n, flags, launches=max(copies, 16))
+        c["batching_speedup_m1_over_m8"] = c["1"]["us_per_row"] / c["8"]["us_per_row"]
+        res[name] = c
+        del pool, w
+    return res
 
 
 def run_e2e(rb, args, world, device):

@@ -98,6 +98,17 @@ mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw
                          uint32_t flags, void *stream);
 
 /*
+ * mrgemv_bf16_plan -- the launch plan mrgemv_bf16_ex would use for (m, n, k,
+ * flags) on a device with sm_count SMs and smem_optin bytes of opt-in shared
+ * memory per block (pure host arithmetic, no CUDA call).  out[8] receives:
+ * grid CTAs, threads per CTA, dynamic shared bytes, weight ring slots, warps
+ * splitting k, column-group warps, row bucket (m rounded up to 1/2/4/8/16),
+ * columns per group.  Size errors are reported as by mrgemv_bf16.
+ */
+mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t flags, int32_t sm_count,
+                           int32_t smem_optin, int32_t *out);
+
+/*
  * router_topk -- per-row top-k of fp32 logits, one CTA per row.
  *
  * The multi-row top-10 launch of Strata PR #109 ("What", router bullet: the

@@ -140,3 +140,42 @@ def test_bounded_wait_selftest_reports_and_context_survives():
     assert mr.mr_poll_errors() == 0
     a, w = synth.router(2)
     check(run_gemv(a, w), a, w)
+
+
+@pytest.mark.parametrize("m", [1, 8, 16])
+def test_sweep_shape_pdl_budget(m):
+    """K=2560, N=6144 under the PDL shared-memory budget: one ring slot, many refills."""
+    a = synth.normal_bits(synth.seed_for(synth.WL_SWEEP, 0), (m, 2560), "bf16", 1.0)
+    w = synth.normal_bits(synth.seed_for(synth.WL_SWEEP, 1), (6144, 2560), "bf16", 1.0 / np.sqrt(2560))
+    c = run_gemv(a, w, flags=mr.MR_GEMV_PDL)
+    check(c, a, w)
+    assert np.array_equal(c.view(np.uint32), run_gemv(a, w).view(np.uint32))
+
+
+def test_back_to_back_pdl_launches_in_a_graph():
+    """Dependent launches overlap; every output must still match its own inputs."""
+    shapes = [(16, 2560, 512), (8, 896, 4864), (1, 2560, 6144), (16, 2560, 6144), (4, 2560, 512)]
+    ins, outs = [], []
+    for i, (m, k, n) in enumerate(shapes):
+        a = synth.normal_bits(700 + i, (m, k), "bf16", 1.0)
+        w = synth.normal_bits(800 + i, (n, k), "bf16", 1.0 / np.sqrt(k))
+        ins.append((a, w, dev_bits(a), dev_bits(w)))
+        outs.append(torch.empty((m, n), dtype=torch.float32, device="cuda"))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for (a, w, A, W), C in zip(ins, outs):
+            mr.mrgemv_bf16(A, W, C, flags=mr.MR_GEMV_PDL)
+    torch.cuda.synchronize()
+    eager = [host(C).copy() for C in outs]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for (a, w, A, W), C in zip(ins, outs):
+            mr.mrgemv_bf16(A, W, C, flags=mr.MR_GEMV_PDL)
+    for C in outs:
+        C.fill_(float("nan"))
+    g.replay()
+    g.replay()
+    for (a, w, _, _), C, e in zip(ins, outs, eager):
+        c = host(C)
+        check(c, a, w)
+        assert np.array_equal(c.view(np.uint32), e.view(np.uint32))

@@ -20,7 +20,7 @@ MR_GEMV_PDL = 0x1
 MR_DEVERR_GEMV_TIMEOUT, MR_DEVERR_GEMM_TIMEOUT, MR_DEVERR_TOPK_TIMEOUT, MR_DEVERR_SELFTEST = 1, 2, 4, 8
 
 EXPORTS = (
-    "mrgemv_bf16", "mrgemv_bf16_ex", "router_topk", "gemm_f16", "gemm_f16_num_tiles",
+    "mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "gemm_f16", "gemm_f16_num_tiles",
     "gemm_f16_tile_name", "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout",
     "mr_status_str", "mr_version",
 )
@@ -33,12 +33,19 @@ class MrError(RuntimeError):
 
 
 def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB):
-        raise ImportError(f"{LIB} is not built; run __graft_entry__.build() (nvcc, sm_100a)")
+    from . import _build
+    if _build.stale():
+        # Sources newer than the library (or no library): compile it now with
+        # nvcc.  Without a toolkit this raises; there is no fallback path.
+        try:
+            _build.build()
+        except Exception as exc:
+            raise ImportError(f"{LIB} is missing or stale and could not be built: {exc}") from exc
     L = ctypes.CDLL(LIB)
     P, I64, I32, U32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32
     L.mrgemv_bf16.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, P]
     L.mrgemv_bf16_ex.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, U32, P]
+    L.mrgemv_bf16_plan.argtypes = [I32, I32, I32, U32, I32, I32, P]
     L.router_topk.argtypes = [P, I64, I32, I32, I32, P, P, I64, P]
     L.gemm_f16.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, I32, I32, P]
     L.gemm_f16_num_tiles.argtypes = []
@@ -51,7 +58,7 @@ def _load() -> ctypes.CDLL:
     L.mr_status_str.restype = ctypes.c_char_p
     L.mr_version.argtypes = []
     L.mr_version.restype = ctypes.c_char_p
-    for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "router_topk", "gemm_f16", "gemm_f16_num_tiles",
+    for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "gemm_f16", "gemm_f16_num_tiles",
                  "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     return L
@@ -104,6 +111,17 @@ def mrgemv_bf16(A, Wt, C, stream=None, flags: int = 0) -> None:
     st = lib.mrgemv_bf16_ex(A.data_ptr(), lda, Wt.data_ptr(), ldw, C.data_ptr(), ldc,
                             m, n, k, flags, _stream(stream))
     _check(st, "mrgemv_bf16")
+
+
+PLAN_FIELDS = ("grid", "threads", "smem_bytes", "ring_slots", "k_warps", "column_warps",
+               "row_bucket", "columns_per_group")
+
+
+def mrgemv_bf16_plan(m: int, n: int, k: int, flags: int, sm_count: int, smem_optin: int) -> dict:
+    """The launch plan of mrgemv_bf16_ex for these sizes on a described device."""
+    out = (ctypes.c_int32 * 8)()
+    _check(lib.mrgemv_bf16_plan(m, n, k, flags, sm_count, smem_optin, out), "mrgemv_bf16_plan")
+    return dict(zip(PLAN_FIELDS, list(out)))
 
 
 def router_topk(logits, topk: int, idx, val=None, stream=None) -> None:

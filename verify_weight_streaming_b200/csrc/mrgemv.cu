@@ -11,10 +11,14 @@
 //    [b*n/G, (b+1)*n/G) of Wt, i.e. a contiguous run of weight rows.
 //  * The block streams through a ring of shared-memory slots, one column group
 //    (up to CG columns x k) per slot, with cp.async.bulk global->shared copies
-//    counted on an mbarrier (no tensor map, no multicast).  The first slots are
+//    counted on an mbarrier (no tensor map, no multicast).  Group g is consumed
+//    by column warp g % CWG from slot g % S; when slots are refilled, S is a
+//    multiple of CWG, so each slot has a single consumer warp that waits for
+//    the slot's successive uses in order.  The first slots are
 //    requested before griddepcontrol.wait, so under programmatic dependent
 //    launch the weight stream overlaps the previous kernel.
-//  * A (m rows, bf16) is staged once in shared memory; rows m..MB-1 are zero.
+//  * A (m rows, bf16) is staged once in shared memory by bulk copies issued
+//    after the grid-dependency wait; rows m..MB-1 are zero.
 //  * Lanes split k in 4-element chunks: chunk q belongs to lane q % 32 of the
 //    k-slice that holds it.  KW warps split k into contiguous slices; KW is a
 //    function of k alone.  Each lane keeps, per (row, column), two fp32
@@ -119,6 +123,7 @@ struct Smem {
     uint64_t *empty;      // [S]
     uint64_t *red_full;   // [CWG]
     uint64_t *red_free;   // [CWG]
+    uint64_t *a_full;     // [1]
     float *red;           // [CWG][KW][32][VPL]
 };
 
@@ -126,11 +131,15 @@ struct Smem {
 template <int MB, int NC, int VPL>
 __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g, int ncol,
                                          int col0, int slice, int cw, int it, int lane,
-                                         int q_begin, int q_end) {
+                                         int q_begin, int q_end, int chunk_groups) {
     const int k = p.k;
     const int slot = g % p.S;
-    const uint32_t par = (uint32_t)(g / p.S) & 1u;
-    if (!mbar_wait_bounded(smem_u32(&sm.full[slot]), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
+    // Without refills (chunk_groups > 0) group g waits on the barrier of the
+    // copy chunk that holds it, phase 0; with refills, on its slot's barrier
+    // for use g / S.
+    const int bar_idx = chunk_groups > 0 ? g / chunk_groups : slot;
+    const uint32_t par = chunk_groups > 0 ? 0u : (uint32_t)(g / p.S) & 1u;
+    if (!mbar_wait_bounded(smem_u32(&sm.full[bar_idx]), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
 
     const uint16_t *w = reinterpret_cast<const uint16_t *>(sm.ring + (size_t)slot * p.slot_bytes);
     float2 acc[MB][NC];
@@ -218,12 +227,13 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
 template <int MB, int NC, int VPL>
 __device__ __forceinline__ bool run_group(const Params &p, const Smem &sm, int g, int ncol,
                                           int col0, int slice, int cw, int it, int lane,
-                                          int q_begin, int q_end) {
+                                          int q_begin, int q_end, int chunk_groups) {
     if constexpr (NC > 1) {
         if (ncol <= NC / 2)
-            return run_group<MB, NC / 2, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end);
+            return run_group<MB, NC / 2, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end,
+                                              chunk_groups);
     }
-    return do_group<MB, NC, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end);
+    return do_group<MB, NC, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end, chunk_groups);
 }
 
 template <int MB, int CG>
@@ -249,7 +259,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     sm.empty = sm.full + p.S;
     sm.red_full = sm.empty + p.S;
     sm.red_free = sm.red_full + p.CWG;
-    sm.red = reinterpret_cast<float *>(sm.red_free + p.CWG);
+    sm.a_full = sm.red_free + p.CWG;
+    sm.red = reinterpret_cast<float *>(sm.a_full + 2);
+
+    // Groups per copy chunk when no slot is refilled (0 when slots are refilled).
+    const int chunk_groups = ng <= p.S ? (int)max(1u, (16384u + p.slot_bytes - 1) / p.slot_bytes) : 0;
 
     auto issue_group = [&](int g) {
         const int slot = g % p.S;
@@ -272,6 +286,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             mbar_init(smem_u32(&sm.full[s]), 1);
             mbar_init(smem_u32(&sm.empty[s]), (uint32_t)p.KW);
         }
+        mbar_init(smem_u32(sm.a_full), 1);
         if (p.KW > 1) {
             for (int c = 0; c < p.CWG; ++c) {
                 mbar_init(smem_u32(&sm.red_full[c]), (uint32_t)(p.KW - 1) * 32u);
@@ -279,25 +294,53 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             }
         }
         fence_mbar_init();
-        const int first = min(ng, p.S);
-        for (int g = 0; g < first; ++g) issue_group(g);
+        if (ng <= p.S) {
+            // Everything fits: copy in chunks of whole groups of >= 16 KB each
+            // (small bulk copies stream far below HBM bandwidth).
+            const uint32_t row_bytes = (uint32_t)k * 2u;
+            for (int c = 0; c * chunk_groups < ng; ++c) {
+                const int g0 = c * chunk_groups;
+                const int cc0 = c_begin + g0 * CG;
+                const int nc = min(chunk_groups * CG, c_end - cc0);
+                const uint32_t bar = smem_u32(&sm.full[c]);
+                const uint32_t dst = smem_u32(sm.ring + (size_t)g0 * p.slot_bytes);
+                mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)nc);
+                if (p.ldw == k) {
+                    bulk_g2s(dst, p.Wt + (int64_t)cc0 * k, row_bytes * (uint32_t)nc, bar);
+                } else {
+                    for (int j = 0; j < nc; ++j)
+                        bulk_g2s(dst + j * row_bytes, p.Wt + (int64_t)(cc0 + j) * p.ldw, row_bytes, bar);
+                }
+            }
+        } else {
+            for (int g = 0; g < p.S; ++g) issue_group(g);
+        }
     }
     // The weight stream is in flight; the next kernel may start launching.
     grid_launch_dependents();
     // A may be produced by the previous kernel on the stream.
     grid_dependency_wait();
 
-    // Stage A (bf16) in shared memory; rows m..MB-1 are zero.
-    {
-        const int chunks = k / 8;  // 16-byte chunks per row
-        for (int e = tid; e < MB * chunks; e += blockDim.x) {
-            const int r = e / chunks, c = e % chunks;
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (r < p.m) val = *reinterpret_cast<const uint4 *>(p.A + (int64_t)r * p.lda + 8 * c);
-            *reinterpret_cast<uint4 *>(sm.a + (size_t)r * k + 8 * c) = val;
+    // Stage A (bf16) in shared memory with bulk copies; rows m..MB-1 are zero.
+    if (tid == 0) {
+        const uint32_t row_bytes = (uint32_t)k * 2u;
+        const uint32_t bar = smem_u32(sm.a_full);
+        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)p.m);
+        if (p.lda == k) {
+            bulk_g2s(smem_u32(sm.a), p.A, row_bytes * (uint32_t)p.m, bar);
+        } else {
+            for (int r = 0; r < p.m; ++r)
+                bulk_g2s(smem_u32(sm.a + (size_t)r * k), p.A + (int64_t)r * p.lda, row_bytes, bar);
         }
     }
+    {
+        const int chunks = k / 8;  // 16-byte chunks per row
+        for (int e = p.m * chunks + tid; e < MB * chunks; e += blockDim.x)
+            *reinterpret_cast<uint4 *>(sm.a + (size_t)(e / chunks) * k + 8 * (e % chunks)) =
+                make_uint4(0u, 0u, 0u, 0u);
+    }
     __syncthreads();
+    if (!mbar_wait_bounded(smem_u32(sm.a_full), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
 
     const int slice = warp % p.KW;
     const int cw = warp / p.KW;
@@ -309,7 +352,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     for (int g = cw; g < ng; g += p.CWG, ++it) {
         const int col0 = c_begin + g * CG;
         const int ncol = min(CG, c_end - col0);
-        const bool ok = run_group<MB, CG, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end);
+        const bool ok =
+            run_group<MB, CG, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end, chunk_groups);
         if (!ok) return;
         // Refill the slot with group g + S once every slice has released it.
         if (slice == 0 && lane == 0 && g + p.S < ng) {
@@ -325,8 +369,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
 
 using KernelFn = void (*)(const Params);
 
+// Columns per group: MB x CG x 2 accumulators per lane stay at 64 registers.
 template <int MB>
-constexpr int col_group() { return MB <= 8 ? 8 : 4; }
+constexpr int col_group() { return MB <= 4 ? 8 : MB == 8 ? 4 : 2; }
+inline int col_group_rt(int MB) { return MB <= 4 ? 8 : MB == 8 ? 4 : 2; }
 
 KernelFn kernel_for(int MB) {
     switch (MB) {
@@ -359,6 +405,86 @@ cudaError_t ensure_attributes(int device) {
 }  // namespace gemv
 }  // namespace mr
 
+namespace mr {
+namespace gemv {
+
+struct Plan {
+    int MB, CG, KW, G, CWG, S;
+    uint32_t a_bytes, slot_bytes;
+    size_t smem;
+};
+
+// Launch plan for (m, n, k) on a device with `sms` SMs and `optin` bytes of
+// opt-in shared memory per block.  Ring invariant: either every column group
+// of a CTA has its own slot (S >= groups, no refills), or S is a multiple of
+// CWG so that slot s is only ever consumed by column warp s % CWG, which waits
+// for the slot's uses strictly in order (a parity wait is then never more
+// than one phase ahead of the barrier).
+mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Plan &pl) {
+    if (m < 1 || n < 1 || k < 8 || sms < 1 || optin < 1) return MR_ERR_INVALID_ARG;
+    if (k % 8 != 0) return MR_ERR_MISALIGNED;
+    if (m > kMaxRows) return MR_ERR_UNSUPPORTED;
+    pl.MB = row_bucket(m);
+    pl.CG = col_group_rt(pl.MB);
+    pl.KW = k_warps(k);
+    pl.G = std::min(sms, n);
+    const int cols_max = (n + pl.G - 1) / pl.G;
+    const int ng_max = (cols_max + pl.CG - 1) / pl.CG;
+    const int cwg0 = std::max(1, std::min(ng_max, kMaxWarps / pl.KW));
+    pl.a_bytes = (uint32_t)(((size_t)pl.MB * k * 2 + 127) / 128 * 128);
+    pl.slot_bytes = (uint32_t)pl.CG * (uint32_t)k * 2u;
+    const size_t vpl = (size_t)std::max(1, pl.MB * pl.CG / 32);
+    const size_t fixed = pl.a_bytes + 16 * (size_t)(2 * ng_max + 2 * cwg0) + 16 +
+                         (size_t)cwg0 * pl.KW * 32 * vpl * 4 + 64;
+    const size_t pdl_budget = 110 * 1024;
+    const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, (size_t)optin) : (size_t)optin;
+    auto slots_for = [&](size_t b) -> int {
+        if (b <= fixed) return 0;
+        return (int)std::min<size_t>((size_t)ng_max, (b - fixed) / pl.slot_bytes);
+    };
+    int s_max = slots_for(budget);
+    if (s_max < 1) s_max = slots_for((size_t)optin);
+    if (s_max < 1) return MR_ERR_UNSUPPORTED;
+    if (s_max < ng_max && s_max < 2 * std::min(cwg0, 2) && budget < (size_t)optin) {
+        // Refills would leave a consumer warp without a second slot: give up
+        // co-residency with the next launch and take the full shared memory.
+        s_max = std::max(s_max, slots_for((size_t)optin));
+    }
+    if (s_max >= ng_max) {
+        pl.S = ng_max;
+        pl.CWG = cwg0;
+    } else {
+        // Each consumer warp gets at least two slots when the budget allows.
+        pl.CWG = std::max(1, std::min(cwg0, s_max / 2));
+        pl.S = (s_max / pl.CWG) * pl.CWG;
+    }
+    pl.smem = pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 16 * (size_t)(pl.S + pl.CWG) + 16 +
+              (size_t)pl.CWG * pl.KW * 32 * vpl * 4;
+    if (pl.smem > (size_t)optin) return MR_ERR_UNSUPPORTED;
+    return MR_OK;
+}
+
+}  // namespace gemv
+}  // namespace mr
+
+extern "C" mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t flags, int32_t sm_count,
+                                      int32_t smem_optin, int32_t *out) {
+    if (!out) return MR_ERR_INVALID_ARG;
+    if (flags & ~MR_GEMV_PDL) return MR_ERR_INVALID_ARG;
+    mr::gemv::Plan pl;
+    const mr_status st = mr::gemv::make_plan(m, n, k, flags, sm_count, smem_optin, pl);
+    if (st != MR_OK) return st;
+    out[0] = pl.G;
+    out[1] = pl.KW * pl.CWG * 32;
+    out[2] = (int32_t)pl.smem;
+    out[3] = pl.S;
+    out[4] = pl.KW;
+    out[5] = pl.CWG;
+    out[6] = pl.MB;
+    out[7] = pl.CG;
+    return MR_OK;
+}
+
 extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw,
                                     float *C, int64_t ldc, int32_t m, int32_t n, int32_t k,
                                     uint32_t flags, void *stream) {
@@ -377,6 +503,9 @@ extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, 
     const int sms = mr_host::sm_count();
     const int optin = mr_host::max_smem_optin();
     if (sms <= 0 || optin <= 0) return MR_ERR_CUDA;
+    Plan pl;
+    const mr_status st = make_plan(m, n, k, flags, sms, optin, pl);
+    if (st != MR_OK) return st;
 
     Params p;
     p.A = static_cast<const uint16_t *>(A);
@@ -388,30 +517,12 @@ extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, 
     p.m = m;
     p.n = n;
     p.k = k;
-    const int MB = row_bucket(m);
-    const int CG = MB <= 8 ? 8 : 4;
-    p.KW = k_warps(k);
-    p.G = std::min(sms, n);
-    const int cols_max = (n + p.G - 1) / p.G;
-    const int ng_max = (cols_max + CG - 1) / CG;
-    p.CWG = std::max(1, std::min(ng_max, kMaxWarps / p.KW));
-    p.a_bytes = (uint32_t)(((size_t)MB * k * 2 + 127) / 128 * 128);
-    p.slot_bytes = (uint32_t)CG * (uint32_t)k * 2u;
-    const int vpl = std::max(1, MB * CG / 32);
-    const size_t fixed = p.a_bytes + 16 * (size_t)(2 * ng_max + 2 * p.CWG) +
-                         (size_t)p.CWG * p.KW * 32 * vpl * 4 + 64;
-    const size_t pdl_budget = 110 * 1024;
-    size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, optin) : (size_t)optin;
-    auto slots_for = [&](size_t b) -> int {
-        if (b <= fixed) return 0;
-        return (int)std::min<size_t>((size_t)ng_max, (b - fixed) / p.slot_bytes);
-    };
-    p.S = slots_for(budget);
-    if (p.S < 1) p.S = slots_for((size_t)optin);
-    if (p.S < 1) return MR_ERR_UNSUPPORTED;
-    const size_t smem = p.a_bytes + (size_t)p.S * p.slot_bytes + 16 * (size_t)(p.S + p.CWG) +
-                        (size_t)p.CWG * p.KW * 32 * vpl * 4;
-    if (smem > (size_t)optin) return MR_ERR_UNSUPPORTED;
+    p.G = pl.G;
+    p.KW = pl.KW;
+    p.CWG = pl.CWG;
+    p.S = pl.S;
+    p.a_bytes = pl.a_bytes;
+    p.slot_bytes = pl.slot_bytes;
 
     e = ensure_attributes(device);
     if (e != cudaSuccess) return mr_host::cuda_status(e);
@@ -419,14 +530,14 @@ extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.G);
     cfg.blockDim = dim3((unsigned)(p.KW * p.CWG * 32));
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = (flags & MR_GEMV_PDL) ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kernel_for(MB), p);
+    e = cudaLaunchKernelEx(&cfg, kernel_for(pl.MB), p);
     return mr_host::cuda_status(e);
 }
 
