@@ -511,12 +511,112 @@ def cpu_baseline(rb):
             "sample": f"{steps} router steps (31 rows each: windows m=1,2,4,8,16, 2560x512, top-10)"}
 
 
+GEMM_M = (150, 192, 306, 448, 700, 1300, 1983, 2048)
+GEMM_N = (512, 640, 1152, 1664, 4096, 6144)
+NARROW_M = (512, 640, 768, 1024, 1983, 2048)
+
+
 def run_gemm_sweep(args):
     import verify_weight_streaming_b200 as mr
     if mr.gemm_f16_num_tiles() <= 0:
         return {"status": "gemm_f16 not built"}
-    from bench_gemm import gemm_sweep  # noqa: E402
     return gemm_sweep(quick=args.quick)
+
+
+def _time_calls(torch, calls, reps=3):
+    """Graph-capture `calls` (a list of thunks), replay, return us per call (min of reps)."""
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for c in calls:
+            c()
+    best = float("inf")
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            g.replay()
+            e1.record(s)
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1) * 1e3 / len(calls))
+    del g
+    return best
+
+
+def gemm_sweep(quick=False):
+    """TFLOP/s of gemm_f16 (auto tile) on the prompt-chunk and narrow shapes.
+
+    Each shape is timed as graph-replayed back-to-back calls that rotate over
+    weight copies (and A copies) whose total exceeds twice the L2, so operands
+    come from HBM as they would for a chunk's successive projections."""
+    import numpy as np
+    import torch
+    import synth
+    import verify_weight_streaming_b200 as mr
+    hbm, tf_burst, tf_sus, kind = load_peaks()
+    props = torch.cuda.get_device_properties(0)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    K = 2560
+    out = {"chunk": {}, "narrow": {}}
+    ms = GEMM_M if not quick else (306, 2048)
+    ns = GEMM_N if not quick else (512, 6144)
+    a_all = torch.from_numpy(synth.chunk(max(ms), 16)[0].view(np.int16)).cuda().view(torch.float16)
+    w_all = torch.from_numpy(synth.chunk(16, max(ns))[1].view(np.int16)).cuda().view(torch.float16)
+    for N in ns:
+        for M in ms:
+            per = (M + N) * K * 2
+            copies = int(min(48, max(2, np.ceil(2.2 * l2 / per))))
+            As = [a_all[:M].clone() for _ in range(copies)]
+            Ws = [w_all[:N].clone() for _ in range(copies)]
+            C = torch.empty((M, N), dtype=torch.float16, device="cuda")
+            calls = [(lambda A=As[i], W=Ws[i]: mr.gemm_f16(A, W, C)) for i in range(copies)]
+            us = _time_calls(torch, calls)
+            tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            out["chunk"][f"{M}x{N}"] = {"us": us, "TFLOPs": tf,
+                                        "tile": mr.gemm_f16_tile_name(mr.gemm_f16_select_tile(M, N, K))}
+            del As, Ws, C
+    big = [v["TFLOPs"] for k, v in out["chunk"].items() if int(k.split("x")[0]) >= 1024]
+    # narrow: one A per M shared by 36 different W[96, 2560]
+    w96 = [torch.from_numpy(synth.narrow(1, w_index=i)[1].view(np.int16)).cuda().view(torch.float16)
+           for i in range(36)]
+    for M in (NARROW_M if not quick else (2048,)):
+        a16 = torch.from_numpy(synth.narrow(M)[0].view(np.int16)).cuda().view(torch.float16)
+        C = torch.empty((M, 96), dtype=torch.float16, device="cuda")
+        calls = [(lambda W=w96[i]: mr.gemm_f16(a16, W, C)) for i in range(36)]
+        us = _time_calls(torch, calls)
+        out["narrow"][str(M)] = {"us_per_call": us, "us_per_36_calls": 36 * us,
+                                 "TFLOPs": 2.0 * M * 96 * K / (us * 1e-6) / 1e12,
+                                 "tile": mr.gemm_f16_tile_name(mr.gemm_f16_select_tile(M, 96, K))}
+    out["summary"] = {"tflops_M_ge_1024_mean": float(np.mean(big)) if big else None,
+                      "tflops_M_ge_1024_max": float(np.max(big)) if big else None,
+                      "peak_bf16_tflops": tf_burst, "peak_kind": kind,
+                      "frac_of_peak_mean": (float(np.mean(big)) / tf_burst) if big else None}
+    return out
+
+
+def gemm_profile_case():
+    """A few GEMM launches on a 2048 x 6144 x 2560 chunk shape (for ncu)."""
+    import numpy as np
+    import torch
+    import synth
+    import verify_weight_streaming_b200 as mr
+    a, w = synth.chunk(2048, 6144)
+    A = torch.from_numpy(a.view(np.int16)).cuda().view(torch.float16)
+    W = torch.from_numpy(w.view(np.int16)).cuda().view(torch.float16)
+    C = torch.empty((2048, 6144), dtype=torch.float16, device="cuda")
+    for _ in range(3):
+        mr.gemm_f16(A, W, C)
+    a, w = synth.narrow(2048)
+    A = torch.from_numpy(a.view(np.int16)).cuda().view(torch.float16)
+    W = torch.from_numpy(w.view(np.int16)).cuda().view(torch.float16)
+    C = torch.empty((2048, 96), dtype=torch.float16, device="cuda")
+    for _ in range(3):
+        mr.gemm_f16(A, W, C)
 
 
 # ------------------------------------------------------------------- profiling
@@ -549,7 +649,6 @@ def profile_case(case: str):
         for _ in range(4):
             mr.router_topk(x, TOPK, idx)
     elif case == "gemm":
-        from bench_gemm import gemm_profile_case
         gemm_profile_case()
     torch.cuda.synchronize()
     assert mr.mr_poll_errors() == 0

@@ -79,3 +79,33 @@ def test_topk_validation(kw, code):
 def test_selftest_limits():
     assert mr.lib.mr_selftest_wait_timeout(0, None) == mr.MR_ERR_INVALID_ARG
     assert mr.lib.mr_selftest_wait_timeout(1000001, None) == mr.MR_ERR_INVALID_ARG
+
+
+def gemm(A=A16, lda=64, W=A16, ldw=64, C=A16, ldc=32, M=4, N=32, K=64, ind=mr.MR_F16, outd=mr.MR_F16, tile=-1):
+    return mr.lib.gemm_f16(A, lda, W, ldw, C, ldc, M, N, K, ind, outd, tile, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(A=None), mr.MR_ERR_INVALID_ARG), (dict(W=None), mr.MR_ERR_INVALID_ARG),
+    (dict(C=None), mr.MR_ERR_INVALID_ARG), (dict(M=0), mr.MR_ERR_INVALID_ARG),
+    (dict(N=0), mr.MR_ERR_INVALID_ARG), (dict(K=0), mr.MR_ERR_INVALID_ARG),
+    (dict(lda=56), mr.MR_ERR_INVALID_ARG), (dict(ldc=24), mr.MR_ERR_INVALID_ARG),
+    (dict(ind=mr.MR_F32), mr.MR_ERR_INVALID_ARG), (dict(outd=7), mr.MR_ERR_INVALID_ARG),
+    (dict(tile=6), mr.MR_ERR_INVALID_ARG), (dict(tile=-2), mr.MR_ERR_INVALID_ARG),
+    (dict(K=60, lda=64, ldw=64), mr.MR_ERR_MISALIGNED), (dict(ldc=36), mr.MR_ERR_MISALIGNED),
+    (dict(C=P(264)), mr.MR_ERR_MISALIGNED), (dict(A=BAD), mr.MR_ERR_MISALIGNED),
+])
+def test_gemm_validation(kw, code):
+    assert gemm(**kw) == code
+
+
+def test_gemm_tiles_and_selector_on_host():
+    n = mr.gemm_f16_num_tiles()
+    assert n == 6
+    names = [mr.gemm_f16_tile_name(t) for t in range(n)]
+    assert names == ["128x32", "128x64", "128x96", "128x128", "128x192", "128x256"]
+    assert mr.gemm_f16_tile_name(n) is None and mr.gemm_f16_tile_name(-1) is None
+    assert mr.gemm_f16_select_tile(0, 96, 2560) == -1
+    for M in (1, 150, 306, 1983, 2048):
+        for N in (1, 96, 512, 6144):
+            assert 0 <= mr.gemm_f16_select_tile(M, N, 2560) < n

@@ -1,10 +1,423 @@
-// gemm_f16: placeholder until the tcgen05 path lands.
+// gemm_f16: C[M,N] = A[M,K] . Wt[N,K]^T on the sm_100a tensor cores.
+//
+// The prompt-chunk GEMM of the "opus r35 track A" audit (section 2, gemm_f16
+// tiles): a family of tile shapes, a selector that is aware of padded tail
+// tiles (M % 128 in 1..64), and outputs that are bitwise identical whatever
+// tile is chosen.  Rebuilt for B200:
+//
+//  * one CTA per 128 x BN output tile, 6 warps: warp 0 issues TMA loads, warp
+//    1 owns the tensor memory and issues tcgen05.mma from one thread, warps
+//    2..5 drain the accumulator (tcgen05.ld) and store the tile;
+//  * A and Wt tiles of 64 K-elements (one 128-byte swizzle atom per row) are
+//    loaded by TMA (no multicast) into a ring of STAGES shared-memory stages,
+//    full/empty mbarriers between the producer and the MMA thread;
+//  * tcgen05.mma.cta_group::1.kind::f16 with M = 128, N = BN, K = 16,
+//    accumulating fp32 in tensor memory.  Every tile runs the same sequence of
+//    K steps (16 at a time, ascending, zero padding past K), with no split-K
+//    or stream-K, so an output element's bits depend on its row of A, its row
+//    of Wt and K only;
+//  * epilogue: fp32 -> f16 / bf16 with round-to-nearest-even (CUDA's
+//    conversion intrinsics), or fp32, stored with the row / column tails masked.
+//  * every wait is bounded; a wait that runs out sets MR_DEVERR_GEMM_TIMEOUT
+//    and the CTA still frees its tensor memory before it exits.
 #include "common.cuh"
 
-extern "C" int32_t gemm_f16_num_tiles(void) { return 0; }
-extern "C" const char *gemm_f16_tile_name(int32_t) { return nullptr; }
-extern "C" int32_t gemm_f16_select_tile(int32_t, int32_t, int32_t) { return -1; }
-extern "C" mr_status gemm_f16(const void *, int64_t, const void *, int64_t, void *, int64_t, int32_t,
-                              int32_t, int32_t, int32_t, int32_t, int32_t, void *) {
-    return MR_ERR_UNSUPPORTED;
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+namespace mr {
+namespace gemm {
+
+constexpr int BM = 128;          // rows per tile (MMA M)
+constexpr int BK = 64;           // K elements per stage (128 bytes of 16-bit data)
+constexpr int kThreads = 192;    // 6 warps
+constexpr uint32_t kABytes = BM * BK * 2;
+
+struct TileDesc {
+    int bn;
+    int stages;
+    int tmem_cols;
+    const char *name;
+};
+
+constexpr TileDesc kTiles[] = {
+    {32, 8, 32, "128x32"},   {64, 8, 64, "128x64"},   {96, 7, 128, "128x96"},
+    {128, 6, 128, "128x128"}, {192, 5, 256, "128x192"}, {256, 4, 256, "128x256"},
+};
+constexpr int kNumTiles = sizeof(kTiles) / sizeof(kTiles[0]);
+
+__host__ __device__ constexpr uint32_t smem_bytes_for(int bn, int stages) {
+    return (uint32_t)stages * (kABytes + (uint32_t)bn * BK * 2) + 1024 /*align*/ + 256 /*barriers*/;
+}
+
+// ---- tcgen05 / TMA PTX wrappers --------------------------------------------
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major operand, 128-byte swizzle:
+// start address >> 4 (bits 0-13), leading byte offset (unused for swizzled
+// K-major, 16 B), stride byte offset = 1024 B between 8-row swizzle atoms
+// (bits 32-45), descriptor version 1 (bits 46-47), layout 128B swizzle = 2
+// (bits 61-63).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)(16u >> 4) << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on `bar` once every tcgen05 operation issued so far by this thread completes.
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// 32 lanes x 32 bits, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---- epilogue stores -----------------------------------------------------
+
+template <int OUT>
+__device__ __forceinline__ void store16(void *C, int64_t ldc, int row, int col, int N, const uint32_t (&r)[16]) {
+    if constexpr (OUT == MR_F32) {
+        float *dst = static_cast<float *>(C) + (int64_t)row * ldc + col;
+        if (col + 16 <= N) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<uint4 *>(dst + i) = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (col + i < N) dst[i] = __uint_as_float(r[i]);
+        }
+    } else {
+        uint32_t h[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float lo = __uint_as_float(r[2 * i]), hi = __uint_as_float(r[2 * i + 1]);
+            if constexpr (OUT == MR_F16) {
+                const __half2 v = __floats2half2_rn(lo, hi);
+                h[i] = *reinterpret_cast<const uint32_t *>(&v);
+            } else {
+                const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+                h[i] = *reinterpret_cast<const uint32_t *>(&v);
+            }
+        }
+        uint16_t *dst = static_cast<uint16_t *>(C) + (int64_t)row * ldc + col;
+        if (col + 16 <= N) {
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(h[4], h[5], h[6], h[7]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (col + i < N) dst[i] = (uint16_t)((i & 1) ? (h[i >> 1] >> 16) : (h[i >> 1] & 0xFFFFu));
+        }
+    }
+}
+
+// ---- the kernel --------------------------------------------------------------
+
+template <int BN, int STAGES, int TMEM_COLS, int OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, void *C,
+                int64_t ldc, int M, int N, int K, uint32_t idesc) {
+    constexpr uint32_t kBBytes = (uint32_t)BN * BK * 2;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+    const uint32_t sA = base;
+    const uint32_t sB = base + STAGES * kABytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + STAGES * (kABytes + kBBytes));
+    uint64_t *full = bars;
+    uint64_t *empty = bars + STAGES;
+    uint64_t *tmem_full = bars + 2 * STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * BM;
+    const int n0 = blockIdx.x * BN;
+    const int nkb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        mbar_init(smem_u32(tmem_full), 1);
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // Producer: stage s is reused after the MMAs reading it complete.
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t par = ((uint32_t)(kb / STAGES) & 1u) ^ 1u;
+                if (!mbar_wait_bounded(smem_u32(&empty[s]), par, MR_DEVERR_GEMM_TIMEOUT)) break;
+                const uint32_t fb = smem_u32(&full[s]);
+                mbar_arrive_expect_tx(fb, kABytes + kBBytes);
+                tma_load_2d(sA + s * kABytes, &tmA, kb * BK, m0, fb);
+                tma_load_2d(sB + s * kBBytes, &tmB, kb * BK, n0, fb);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            bool ok = true;
+            for (int kb = 0; kb < nkb && ok; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t par = (uint32_t)(kb / STAGES) & 1u;
+                ok = mbar_wait_bounded(smem_u32(&full[s]), par, MR_DEVERR_GEMM_TIMEOUT);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint64_t ad = sw128_desc(sA + s * kABytes + kk * 32);
+                    const uint64_t bd = sw128_desc(sB + s * kBBytes + kk * 32);
+                    mma_f16(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                }
+                mma_commit(smem_u32(&empty[s]));
+            }
+            if (ok) mma_commit(smem_u32(tmem_full));
+        }
+    } else {
+        // Epilogue warps 2..5: warp w reads tensor-memory lanes 32*(w%4) .. +31.
+        const int q = warp & 3;
+        const int row = m0 + 32 * q + lane;
+        const bool ok = mbar_wait_bounded(smem_u32(tmem_full), 0u, MR_DEVERR_GEMM_TIMEOUT);
+        tc_fence_after();
+        if (ok) {
+#pragma unroll 1
+            for (int c = 0; c < BN / 16; ++c) {
+                uint32_t r[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * 16), r);
+                const int col = n0 + c * 16;
+                if (row < M && col < N) store16<OUT>(C, ldc, row, col, N, r);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ---- host side -------------------------------------------------------------
+
+using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, void *, int64_t, int, int, int, uint32_t);
+
+template <int T, int OUT>
+constexpr KernelFn kernel_of() {
+    return gemm_kernel<kTiles[T].bn, kTiles[T].stages, kTiles[T].tmem_cols, OUT>;
+}
+
+template <int OUT>
+KernelFn pick_out(int t) {
+    switch (t) {
+        case 0: return kernel_of<0, OUT>();
+        case 1: return kernel_of<1, OUT>();
+        case 2: return kernel_of<2, OUT>();
+        case 3: return kernel_of<3, OUT>();
+        case 4: return kernel_of<4, OUT>();
+        default: return kernel_of<5, OUT>();
+    }
+}
+
+KernelFn kernel_for(int tile, int out) {
+    if (out == MR_F16) return pick_out<MR_F16>(tile);
+    if (out == MR_BF16) return pick_out<MR_BF16>(tile);
+    return pick_out<MR_F32>(tile);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_mutex;
+bool g_attr_done[64] = {};
+
+cudaError_t init_device(int device) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (device >= 0 && device < 64 && !g_attr_done[device]) {
+        for (int t = 0; t < kNumTiles; ++t)
+            for (int out = 0; out < 3; ++out) {
+                cudaError_t e = cudaFuncSetAttribute(kernel_for(t, out), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)smem_bytes_for(kTiles[t].bn, kTiles[t].stages));
+                if (e != cudaSuccess) return e;
+            }
+        g_attr_done[device] = true;
+    }
+    return cudaSuccess;
+}
+
+bool encode_operand(CUtensorMap *map, const void *ptr, int64_t rows, int64_t cols, int64_t ld, int dtype,
+                    int box_rows) {
+    const CUtensorMapDataType dt =
+        dtype == MR_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), A and B
+// formats (bits 7-9, 10-12: 0 = f16, 1 = bf16), both K-major (bits 15, 16 = 0),
+// N >> 3 (bits 17-22), M >> 4 (bits 24-28).
+uint32_t make_idesc(int in_dtype, int bn) {
+    const uint32_t fmt = in_dtype == MR_BF16 ? 1u : 0u;
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+// Tile selection: estimated time = waves x per-tile time, where a wave is one
+// CTA per SM, per-tile time is the padded MMA work of the tile at a rate that
+// grows with BN (wider tiles reuse each A stage for more columns) plus a fixed
+// prologue / epilogue cost.  Row tails are counted as whole 128-row tiles, so
+// an M whose M % 128 is small pays for the padding it creates; narrow N (the
+// N = 96 projections) favours tiles that divide N and spread over more SMs.
+int select_tile(int M, int N, int K, int sms) {
+    if (M < 1 || N < 1 || K < 1 || sms < 1) return -1;
+    const double eff[kNumTiles] = {0.30, 0.55, 0.70, 0.80, 0.88, 0.92};
+    const double per_sm_flops_us = 1.6e15 / 148.0 * 1e-6;   // dense f16 per SM per microsecond
+    int best = -1;
+    double best_t = 1e300;
+    for (int t = 0; t < kNumTiles; ++t) {
+        const int bn = kTiles[t].bn;
+        const int64_t tiles = (int64_t)((M + BM - 1) / BM) * ((N + bn - 1) / bn);
+        const int64_t waves = (tiles + sms - 1) / sms;
+        const double kpad = (double)((K + BK - 1) / BK * BK);
+        const double tile_us = 2.0 * BM * bn * kpad / (per_sm_flops_us * eff[t]) + 1.5;
+        // A tile streamed per CTA bounds narrow tiles: bytes per CTA at ~150 GB/s.
+        const double stream_us = (BM + bn) * kpad * 2.0 / 150e3;
+        const double t_est = (double)waves * std::max(tile_us, stream_us);
+        if (t_est < best_t * 0.999) {
+            best_t = t_est;
+            best = t;
+        }
+    }
+    return best;
+}
+
+}  // namespace gemm
+}  // namespace mr
+
+extern "C" int32_t gemm_f16_num_tiles(void) { return mr::gemm::kNumTiles; }
+
+extern "C" const char *gemm_f16_tile_name(int32_t tile_id) {
+    if (tile_id < 0 || tile_id >= mr::gemm::kNumTiles) return nullptr;
+    return mr::gemm::kTiles[tile_id].name;
+}
+
+extern "C" int32_t gemm_f16_select_tile(int32_t M, int32_t N, int32_t K) {
+    int sms = mr_host::sm_count();
+    if (sms <= 0) sms = 148;
+    return mr::gemm::select_tile(M, N, K, sms);
+}
+
+extern "C" mr_status gemm_f16(const void *A, int64_t lda, const void *Wt, int64_t ldw, void *C, int64_t ldc,
+                              int32_t M, int32_t N, int32_t K, int32_t in_dtype, int32_t out_dtype, int32_t tile_id,
+                              void *stream) {
+    using namespace mr::gemm;
+    if (!A || !Wt || !C) return MR_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < 1) return MR_ERR_INVALID_ARG;
+    if (lda < K || ldw < K || ldc < N) return MR_ERR_INVALID_ARG;
+    if (in_dtype != MR_F16 && in_dtype != MR_BF16) return MR_ERR_INVALID_ARG;
+    if (out_dtype != MR_F16 && out_dtype != MR_BF16 && out_dtype != MR_F32) return MR_ERR_INVALID_ARG;
+    if (tile_id < -1 || tile_id >= kNumTiles) return MR_ERR_INVALID_ARG;
+    if (K % 8 != 0 || lda % 8 != 0 || ldw % 8 != 0 || ldc % 8 != 0) return MR_ERR_MISALIGNED;
+    if (((uintptr_t)A & 15u) || ((uintptr_t)Wt & 15u) || ((uintptr_t)C & 15u)) return MR_ERR_MISALIGNED;
+
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) return mr_host::cuda_status(e);
+    e = init_device(device);
+    if (e != cudaSuccess) return MR_ERR_CUDA;
+    const int sms = mr_host::sm_count();
+    const int t = tile_id >= 0 ? tile_id : select_tile(M, N, K, sms > 0 ? sms : 148);
+    if (t < 0) return MR_ERR_INVALID_ARG;
+    const TileDesc &td = kTiles[t];
+
+    CUtensorMap ta, tb;
+    if (!encode_operand(&ta, A, M, K, lda, in_dtype, BM)) return MR_ERR_CUDA;
+    if (!encode_operand(&tb, Wt, N, K, ldw, in_dtype, td.bn)) return MR_ERR_CUDA;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((N + td.bn - 1) / td.bn), (unsigned)((M + BM - 1) / BM));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem_bytes_for(td.bn, td.stages);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    e = cudaLaunchKernelEx(&cfg, kernel_for(t, out_dtype), ta, tb, C, ldc, (int)M, (int)N, (int)K,
+                           make_idesc(in_dtype, td.bn));
+    return mr_host::cuda_status(e);
 }
