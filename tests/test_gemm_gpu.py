@@ -37,7 +37,7 @@ def run_gemm(a_bits, w_bits, in_fmt="f16", out_fmt="f16", tile=-1, ldc=None, lda
         buf[:, :K] = A
         A = buf[:, :K]
     W = dev_bits(w_bits, TORCH_DT[in_fmt])
-    ldc = ldc or N
+    ldc = ldc or (N + 7) // 8 * 8
     cbuf = torch.full((M + 1, ldc), float("nan"), dtype=TORCH_DT[out_fmt], device="cuda")
     C = cbuf[:M, :N]
     mr.gemm_f16(A, W, C, tile_id=tile)
