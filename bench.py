@@ -637,12 +637,15 @@ def profile_case(case: str):
             C = torch.empty((m, N_ROUTER), dtype=torch.float32, device="cuda")
             for i in range(4):
                 mr.mrgemv_bf16(A[:m], pool[(7 * i + m) % len(pool)], C)
-        a16, w16 = synth.gemv_ffn(8)
+    elif case in ("gemv_ffn", "gemv_sweep"):
+        k, n, wl, m = (896, 4864, synth.WL_GEMV_FFN, 16) if case == "gemv_ffn" else (2560, 6144, synth.WL_SWEEP, 8)
+        a16 = synth.normal_bits(synth.seed_for(wl, 0), (16, k), "bf16", 1.0)
+        w16 = synth.normal_bits(synth.seed_for(wl, 1), (n, k), "bf16", 1.0 / np.sqrt(k))
+        W = [torch.from_numpy(w16.view(np.int16)).cuda() for _ in range(8)]
         A = torch.from_numpy(a16.view(np.int16)).cuda()
-        W = [torch.from_numpy(w16.view(np.int16)).cuda() for _ in range(30)]
-        C = torch.empty((8, 4864), dtype=torch.float32, device="cuda")
-        for i in range(4):
-            mr.mrgemv_bf16(A, W[(5 * i) % 30], C)
+        C = torch.empty((m, n), dtype=torch.float32, device="cuda")
+        for i in range(3):
+            mr.mrgemv_bf16(A[:m], W[i], C)
     elif case == "topk":
         x = torch.randn(16, 512, device="cuda")
         idx = torch.empty((16, TOPK), dtype=torch.int32, device="cuda")
