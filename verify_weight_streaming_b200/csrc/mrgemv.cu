@@ -21,10 +21,11 @@
 //    after the grid-dependency wait; rows m..MB-1 are zero.
 //  * Lanes split k in 4-element chunks: chunk q belongs to lane q % 32 of the
 //    k-slice that holds it.  KW warps split k into contiguous slices; KW is a
-//    function of k alone.  Each lane keeps, per (row, column), two fp32
-//    accumulators (even / odd element of each pair) updated with
-//    fma.rn.f32x2 in ascending chunk order.
-//  * Reduction: even + odd, then a fixed xor-butterfly over the 32 lanes
+//    function of k alone.  Each lane keeps one fp32 accumulator per (row,
+//    column), updated in ascending k; rows are paired so that one
+//    fma.rn.f32x2 advances two rows' chains (a single row runs with a zero
+//    partner row).
+//  * Reduction: a fixed xor-butterfly over the 32 lanes
 //    (bit 16, 8, 4, 2, 1; realised as a reduce-scatter so each lane finishes a
 //    share of the values), then the KW slices in slice order.  The tree of
 //    every output element is the same for every m, every row position and
@@ -70,16 +71,27 @@ __host__ __device__ inline int k_warps(int k) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// acc.x = fma(a.x, b.x, acc.x); acc.y = fma(a.y, b.y, acc.y), both round-to-nearest.
-__device__ __forceinline__ void ffma2(float2 &acc, float ax, float ay, float bx, float by) {
-    asm("{\n\t.reg .b64 a2, b2, c2;\n\t"
-        "mov.b64 a2, {%2, %3};\n\t"
-        "mov.b64 b2, {%4, %5};\n\t"
-        "mov.b64 c2, {%0, %1};\n\t"
-        "fma.rn.f32x2 c2, a2, b2, c2;\n\t"
-        "mov.b64 {%0, %1}, c2;\n\t}"
-        : "+f"(acc.x), "+f"(acc.y)
-        : "f"(ax), "f"(ay), "f"(bx), "f"(by));
+// Packed pairs of fp32 in one 64-bit register pair (low half first).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float lo_of(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo;
+}
+__device__ __forceinline__ float hi_of(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return hi;
+}
+
+// acc.lo = fma(a.lo, b.lo, acc.lo); acc.hi = fma(a.hi, b.hi, acc.hi): two
+// independent round-to-nearest fp32 FMAs in one instruction.
+__device__ __forceinline__ void ffma2(uint64_t &acc, uint64_t a, uint64_t b) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
 }
 
 // Reduce-scatter over the warp: level D pairs lanes that differ in bit D (16,
@@ -142,32 +154,41 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     if (!mbar_wait_bounded(smem_u32(&sm.full[bar_idx]), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
 
     const uint16_t *w = reinterpret_cast<const uint16_t *>(sm.ring + (size_t)slot * p.slot_bytes);
-    float2 acc[MB][NC];
+    // acc[rp][j] holds rows (2rp, 2rp+1) of column j: one fp32 chain per
+    // (row, column), over this lane's k positions in ascending order.
+    constexpr int RP = MB / 2;
+    uint64_t acc[RP][NC];
 #pragma unroll
-    for (int r = 0; r < MB; ++r)
+    for (int rp = 0; rp < RP; ++rp)
 #pragma unroll
-        for (int j = 0; j < NC; ++j) acc[r][j] = make_float2(0.f, 0.f);
+        for (int j = 0; j < NC; ++j) acc[rp][j] = 0ull;
 
 #pragma unroll 2
     for (int q = q_begin + lane; q < q_end; q += 32) {
-        float w0[NC], w1[NC], w2[NC], w3[NC];
+        uint64_t wd[4][NC];  // (w, w) for element e of the chunk, column j
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
             const uint2 raw = *reinterpret_cast<const uint2 *>(w + (size_t)j * k + 4 * q);
-            w0[j] = bf16lo(raw.x);
-            w1[j] = bf16hi(raw.x);
-            w2[j] = bf16lo(raw.y);
-            w3[j] = bf16hi(raw.y);
+            const float w0 = bf16lo(raw.x), w1 = bf16hi(raw.x), w2 = bf16lo(raw.y), w3 = bf16hi(raw.y);
+            wd[0][j] = pack2(w0, w0);
+            wd[1][j] = pack2(w1, w1);
+            wd[2][j] = pack2(w2, w2);
+            wd[3][j] = pack2(w3, w3);
         }
 #pragma unroll
-        for (int r = 0; r < MB; ++r) {
-            const uint2 ar = *reinterpret_cast<const uint2 *>(sm.a + (size_t)r * k + 4 * q);
-            const float a0 = bf16lo(ar.x), a1 = bf16hi(ar.x);
-            const float a2 = bf16lo(ar.y), a3 = bf16hi(ar.y);
+        for (int rp = 0; rp < RP; ++rp) {
+            const uint2 r0 = *reinterpret_cast<const uint2 *>(sm.a + (size_t)(2 * rp) * k + 4 * q);
+            const uint2 r1 = *reinterpret_cast<const uint2 *>(sm.a + (size_t)(2 * rp + 1) * k + 4 * q);
+            const uint64_t a0 = pack2(bf16lo(r0.x), bf16lo(r1.x));
+            const uint64_t a1 = pack2(bf16hi(r0.x), bf16hi(r1.x));
+            const uint64_t a2 = pack2(bf16lo(r0.y), bf16lo(r1.y));
+            const uint64_t a3 = pack2(bf16hi(r0.y), bf16hi(r1.y));
 #pragma unroll
             for (int j = 0; j < NC; ++j) {
-                ffma2(acc[r][j], a0, a1, w0[j], w1[j]);
-                ffma2(acc[r][j], a2, a3, w2[j], w3[j]);
+                ffma2(acc[rp][j], a0, wd[0][j]);
+                ffma2(acc[rp][j], a1, wd[1][j]);
+                ffma2(acc[rp][j], a2, wd[2][j]);
+                ffma2(acc[rp][j], a3, wd[3][j]);
             }
         }
     }
@@ -178,9 +199,12 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     constexpr int V = MB * NC;
     float v[V];
 #pragma unroll
-    for (int r = 0; r < MB; ++r)
+    for (int rp = 0; rp < RP; ++rp)
 #pragma unroll
-        for (int j = 0; j < NC; ++j) v[r * NC + j] = __fadd_rn(acc[r][j].x, acc[r][j].y);
+        for (int j = 0; j < NC; ++j) {
+            v[(2 * rp) * NC + j] = lo_of(acc[rp][j]);
+            v[(2 * rp + 1) * NC + j] = hi_of(acc[rp][j]);
+        }
     int base = 0;
     ReduceScatter<V, 16>::run(v, lane, base);
     constexpr int PL = Scatter<V>::kPerLane;
@@ -369,14 +393,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
 
 using KernelFn = void (*)(const Params);
 
-// Columns per group: MB x CG x 2 accumulators per lane stay at 64 registers.
+// Columns per group: at most 64 fp32 accumulators per lane (MB x CG).
 template <int MB>
-constexpr int col_group() { return MB <= 4 ? 8 : MB == 8 ? 4 : 2; }
-inline int col_group_rt(int MB) { return MB <= 4 ? 8 : MB == 8 ? 4 : 2; }
+constexpr int col_group() { return MB <= 8 ? 8 : 4; }
+inline int col_group_rt(int MB) { return MB <= 8 ? 8 : 4; }
 
 KernelFn kernel_for(int MB) {
     switch (MB) {
-        case 1: return gemv_kernel<1, col_group<1>()>;
         case 2: return gemv_kernel<2, col_group<2>()>;
         case 4: return gemv_kernel<4, col_group<4>()>;
         case 8: return gemv_kernel<8, col_group<8>()>;
@@ -384,7 +407,8 @@ KernelFn kernel_for(int MB) {
     }
 }
 
-int row_bucket(int m) { return m <= 1 ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
+// Rows are processed in pairs, so a single row runs in the 2-row kernel with a zero second row.
+int row_bucket(int m) { return m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
 
 std::mutex g_attr_mutex;
 bool g_attr_done[64] = {};
@@ -393,7 +417,7 @@ cudaError_t ensure_attributes(int device) {
     std::lock_guard<std::mutex> lock(g_attr_mutex);
     if (device >= 0 && device < 64 && g_attr_done[device]) return cudaSuccess;
     const int optin = mr_host::max_smem_optin();
-    const int mbs[] = {1, 2, 4, 8, 16};
+    const int mbs[] = {2, 4, 8, 16};
     for (int mb : mbs) {
         cudaError_t e = cudaFuncSetAttribute(kernel_for(mb), cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
         if (e != cudaSuccess) return e;
