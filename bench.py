@@ -2,8 +2,9 @@
 
 One step = one pass of the router hot path over one batch: for each window
 size m in (1, 2, 4, 8, 16), A[m,2560] bf16 x W_r[2560,512] bf16 -> fp32 logits
-(mrgemv_bf16, weight streamed once) -> per-row top-10 (router_topk).  That is
-31 rows and 10 kernel launches per step.  The weight comes from a rotating pool
+(weight streamed once) -> per-row top-10, in one fused launch per window
+(router_gemv_topk).  That is 31 rows and 5 kernel launches per step; the
+two-launch form (mrgemv_bf16 then router_topk) is timed alongside.  The weight comes from a rotating pool
 of copies larger than twice the L2, so every launch reads it from HBM.
 
 Printed (rank 0, one JSON line): us_per_row over the whole step (lower is
@@ -269,29 +270,37 @@ class RouterBench:
         self.val = {m: torch.empty((m, TOPK), dtype=torch.float32, device=device) for m in WINDOWS}
         self.stream = torch.cuda.Stream(device)
         self.cursor = 0
+        nbytes = mr.router_gemv_topk_workspace_bytes(16, N_ROUTER, False)
+        self.ws = torch.zeros((nbytes + 3) // 4, dtype=torch.int32, device=device)
 
     def _next_w(self):
         w = self.W[self.cursor % self.pool]
         self.cursor += 1
         return w
 
-    def step(self, flags):
+    def step(self, flags, fused=True):
+        """One router step: for each window size, GEMV + top-10 (one fused launch,
+        or the two-launch form mrgemv_bf16 then router_topk)."""
         mr = self.mr
         for m in WINDOWS:
-            mr.mrgemv_bf16(self.A[:m], self._next_w(), self.C[m], flags=flags)
-            mr.router_topk(self.C[m], TOPK, self.idx[m], self.val[m])
+            if fused:
+                mr.router_gemv_topk(self.A[:m], self._next_w(), TOPK, self.idx[m], self.val[m],
+                                    workspace=self.ws, flags=flags)
+            else:
+                mr.mrgemv_bf16(self.A[:m], self._next_w(), self.C[m], flags=flags)
+                mr.router_topk(self.C[m], TOPK, self.idx[m], self.val[m])
 
-    def capture_steps(self, count, flags):
+    def capture_steps(self, count, flags, fused=True):
         """One CUDA graph per step, each with its own slice of the weight pool."""
         torch = self.torch
         graphs = []
         with torch.cuda.stream(self.stream):
-            self.step(flags)  # warm the launch path outside capture
+            self.step(flags, fused)  # warm the launch path outside capture
         torch.cuda.synchronize()
         for _ in range(count):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=self.stream):
-                self.step(flags)
+                self.step(flags, fused)
             graphs.append(g)
         return graphs
 
@@ -346,6 +355,11 @@ def run_gpu(args, world, rank, local):
     # whole-job time per row: all ranks' rows over the slowest rank's time
     us_per_row = elapsed_max / (args.steps * step_rows() * world)
     clocks = clk.summary()
+    # the same step with the two-launch router (GEMV, then top-k), for comparison
+    graphs2 = rb.capture_steps(steps_per_cycle, flags, fused=False)
+    rb.time_graphs(graphs2, 3)
+    two_launch_us = max_over_ranks(rb.time_graphs(graphs2, args.steps), world, device)
+    del graphs2
     clocks["sampled_over_us"] = elapsed_us + sum(extra)
 
     # ---- per-m curve and the GEMV roofline (back-to-back graph-captured calls)
@@ -379,7 +393,8 @@ def run_gpu(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": elapsed_max / args.steps / 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(), "gpu_launches": args.steps * 2 * len(WINDOWS),
+            "config": workload_config(), "gpu_launches": args.steps * len(WINDOWS),
+            "two_launch_us_per_row": two_launch_us / (args.steps * step_rows() * world),
             "device_errors": errs, "clocks": clocks, "roofline": roofline,
             "curve": {"router": curve, "batching_speedup_m1_over_m8": speedup, **extra_curves},
             "e2e": e2e, "gemm": gemm, "cpu_baseline": cpu,
@@ -473,8 +488,8 @@ def run_e2e(rb, args, world, device):
     def one_step():
         for m in WINDOWS:
             a_dev[m].copy_(a_host[:m], non_blocking=True)
-            mr.mrgemv_bf16(a_dev[m], rb._next_w(), rb.C[m], flags=flags)
-            mr.router_topk(rb.C[m], TOPK, rb.idx[m], rb.val[m])
+            mr.router_gemv_topk(a_dev[m], rb._next_w(), TOPK, rb.idx[m], rb.val[m], workspace=rb.ws,
+                                flags=flags)
             idx_host[m].copy_(rb.idx[m], non_blocking=True)
             val_host[m].copy_(rb.val[m], non_blocking=True)
 
@@ -495,7 +510,7 @@ def run_e2e(rb, args, world, device):
     d2h = sum(m * TOPK * 8 for m in WINDOWS)
     return {"value": us / (steps * step_rows() * world), "unit": "us/row",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "api": "verify_weight_streaming_b200.mrgemv_bf16 + router_topk, pinned host buffers"}
+            "api": "verify_weight_streaming_b200.router_gemv_topk, pinned host buffers"}
 
 
 def cpu_baseline(rb):

@@ -34,6 +34,7 @@
 #ifndef MRGEMM_H
 #define MRGEMM_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -107,6 +108,34 @@ mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw
  */
 mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t flags, int32_t sm_count,
                            int32_t smem_optin, int32_t *out);
+
+/*
+ * router_gemv_topk -- the router in one launch: the multi-row GEMV of
+ * mrgemv_bf16 followed by the per-row top-k of router_topk.  The two steps of
+ * Strata PR #109 ("What", router bullet: one multi-row GEMV plus one multi-row
+ * top-10 launch) are fused: the CTA that stores its logits last (an atomic
+ * ticket in the workspace) selects the top-k of every row.  idx / val are
+ * bitwise the outputs of mrgemv_bf16 then router_topk on the same inputs.
+ *
+ * A, Wt, m, n, k, lda, ldw, flags : as mrgemv_bf16_ex.
+ * logits : NULL, or m rows of n fp32 (row stride ldl >= n) that receive the
+ *          GEMV output.  When NULL the logits live in the workspace.
+ * topk, idx, val, ldo : as router_topk (val may be NULL).
+ * workspace : device memory, 256-byte aligned, of at least
+ *          router_gemv_topk_workspace_bytes(m, n, logits != NULL) bytes.
+ *          Its first MR_ROUTER_TICKET_BYTES must be zero before the first
+ *          call; every completed call leaves them zero again.  Calls that may
+ *          run at the same time (other streams) need separate workspaces.
+ */
+#define MR_ROUTER_TICKET_BYTES 256u
+mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt, int64_t ldw,
+                           float *logits, int64_t ldl, int32_t m, int32_t n, int32_t k,
+                           int32_t topk, int32_t *idx, float *val, int64_t ldo,
+                           void *workspace, size_t workspace_bytes, uint32_t flags,
+                           void *stream);
+
+/* Workspace bytes router_gemv_topk needs (0 for invalid sizes). */
+size_t router_gemv_topk_workspace_bytes(int32_t m, int32_t n, int32_t logits_provided);
 
 /*
  * router_topk -- per-row top-k of fp32 logits, one CTA per row.

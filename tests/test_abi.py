@@ -109,3 +109,25 @@ def test_gemm_tiles_and_selector_on_host():
     for M in (1, 150, 306, 1983, 2048):
         for N in (1, 96, 512, 6144):
             assert 0 <= mr.gemm_f16_select_tile(M, N, 2560) < n
+
+
+def fused(A=A16, W=A16, logits=None, m=4, n=512, k=64, topk=10, idx=A16, ldo=10, ws=P(512), wsb=1 << 20):
+    return mr.lib.router_gemv_topk(A, 64, W, 64, logits, 512, m, n, k, topk, idx, None, ldo, ws, wsb, 0, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=None), mr.MR_ERR_INVALID_ARG), (dict(idx=None), mr.MR_ERR_INVALID_ARG),
+    (dict(topk=0), mr.MR_ERR_INVALID_ARG), (dict(topk=11), mr.MR_ERR_INVALID_ARG),
+    (dict(topk=33, ldo=33), mr.MR_ERR_UNSUPPORTED), (dict(ws=P(272)), mr.MR_ERR_MISALIGNED),
+    (dict(wsb=255), mr.MR_ERR_INVALID_ARG), (dict(wsb=256), mr.MR_ERR_INVALID_ARG),
+    (dict(m=17), mr.MR_ERR_UNSUPPORTED), (dict(A=None), mr.MR_ERR_INVALID_ARG),
+])
+def test_fused_router_validation(kw, code):
+    assert fused(**kw) == code
+
+
+def test_fused_router_workspace_bytes():
+    assert mr.router_gemv_topk_workspace_bytes(4, 512, True) == 256
+    assert mr.router_gemv_topk_workspace_bytes(4, 512, False) == 256 + 4 * 512 * 4
+    assert mr.router_gemv_topk_workspace_bytes(0, 512, False) == 0
+    assert fused(logits=P(1024), wsb=256) == mr.MR_ERR_CUDA  # valid; no device here

@@ -1,0 +1,105 @@
+"""router_gemv_topk (GEMV + top-k in one launch) against the two-launch path:
+logits, indices and values bitwise equal; the ticket returns to zero."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import dev_bits, host, need_gpu, torch
+
+import verify_weight_streaming_b200 as mr
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+    yield
+    assert mr.mr_poll_errors() == 0
+
+
+def workspace(m, n, with_logits):
+    nbytes = mr.router_gemv_topk_workspace_bytes(m, n, with_logits)
+    return torch.zeros((nbytes + 3) // 4, dtype=torch.int32, device="cuda")
+
+
+def two_launch(A, W, m, n, topk):
+    C = torch.empty((m, n), dtype=torch.float32, device="cuda")
+    idx = torch.empty((m, topk), dtype=torch.int32, device="cuda")
+    val = torch.empty((m, topk), dtype=torch.float32, device="cuda")
+    mr.mrgemv_bf16(A, W, C)
+    mr.router_topk(C, topk, idx, val)
+    return host(C), host(idx), host(val)
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 8, 16])
+@pytest.mark.parametrize("with_logits", [True, False])
+def test_fused_matches_two_launches(m, with_logits):
+    a, w = synth.router(m)
+    A, W = dev_bits(a), dev_bits(w)
+    c_ref, i_ref, v_ref = two_launch(A, W, m, 512, 10)
+    ws = workspace(m, 512, with_logits)
+    idx = torch.full((m, 10), -1, dtype=torch.int32, device="cuda")
+    val = torch.full((m, 10), float("nan"), dtype=torch.float32, device="cuda")
+    logits = torch.empty((m, 512), dtype=torch.float32, device="cuda") if with_logits else None
+    mr.router_gemv_topk(A, W, 10, idx, val, logits=logits, workspace=ws)
+    assert np.array_equal(host(idx), i_ref)
+    assert np.array_equal(host(val).view(np.uint32), v_ref.view(np.uint32))
+    if with_logits:
+        assert np.array_equal(host(logits).view(np.uint32), c_ref.view(np.uint32))
+    assert int(host(ws)[0]) == 0, "ticket not returned to zero"
+    ri, _ = oracle.topk(c_ref, 10)
+    assert np.array_equal(host(idx), ri)
+
+
+@pytest.mark.parametrize("m,n,k,topk", [(5, 37, 136, 7), (16, 4864, 896, 32), (2, 6144, 2560, 10),
+                                        (9, 3, 8, 3), (16, 149, 1024, 1)])
+def test_other_shapes(m, n, k, topk):
+    a = synth.normal_bits(500 + n, (m, k), "bf16", 1.0)
+    w = synth.normal_bits(600 + k, (n, k), "bf16", 1.0 / np.sqrt(k))
+    A, W = dev_bits(a), dev_bits(w)
+    c_ref, i_ref, v_ref = two_launch(A, W, m, n, topk)
+    ws = workspace(m, n, False)
+    idx = torch.empty((m, topk), dtype=torch.int32, device="cuda")
+    val = torch.empty((m, topk), dtype=torch.float32, device="cuda")
+    mr.router_gemv_topk(A, W, topk, idx, val, workspace=ws)
+    assert np.array_equal(host(idx), i_ref)
+    assert np.array_equal(host(val).view(np.uint32), v_ref.view(np.uint32))
+    c64, s64 = oracle.matmul(a, "bf16", w, "bf16")
+    ok, worst, _ = oracle.check_matmul(c_ref, c64, s64)
+    assert ok, worst
+
+
+def test_many_calls_graph_and_pdl_reuse_one_workspace():
+    ms = [16, 1, 8, 4, 2]
+    ins = []
+    for i, m in enumerate(ms):
+        a = synth.normal_bits(900 + i, (m, 2560), "bf16", 1.0)
+        w = synth.normal_bits(950 + i, (512, 2560), "bf16", 0.02)
+        ins.append((m, dev_bits(a), dev_bits(w)))
+    refs = [two_launch(A, W, m, 512, 10) for m, A, W in ins]
+    ws = workspace(16, 512, False)
+    outs = [(torch.empty((m, 10), dtype=torch.int32, device="cuda"),
+             torch.empty((m, 10), dtype=torch.float32, device="cuda")) for m, _, _ in ins]
+    s = torch.cuda.Stream()
+    for _ in range(20):
+        with torch.cuda.stream(s):
+            for (m, A, W), (i, v) in zip(ins, outs):
+                mr.router_gemv_topk(A, W, 10, i, v, workspace=ws, flags=mr.MR_GEMV_PDL)
+    torch.cuda.synchronize()
+    for (c, ir, vr), (i, v) in zip(refs, outs):
+        assert np.array_equal(host(i), ir)
+        assert np.array_equal(host(v).view(np.uint32), vr.view(np.uint32))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for (m, A, W), (i, v) in zip(ins, outs):
+            mr.router_gemv_topk(A, W, 10, i, v, workspace=ws, flags=mr.MR_GEMV_PDL)
+    for i, v in outs:
+        i.fill_(-1)
+    for _ in range(10):
+        g.replay()
+    torch.cuda.synchronize()
+    for (c, ir, vr), (i, v) in zip(refs, outs):
+        assert np.array_equal(host(i), ir)
+    assert int(host(ws)[0]) == 0

@@ -20,7 +20,8 @@ MR_GEMV_PDL = 0x1
 MR_DEVERR_GEMV_TIMEOUT, MR_DEVERR_GEMM_TIMEOUT, MR_DEVERR_TOPK_TIMEOUT, MR_DEVERR_SELFTEST = 1, 2, 4, 8
 
 EXPORTS = (
-    "mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "gemm_f16", "gemm_f16_num_tiles",
+    "mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
+    "router_gemv_topk_workspace_bytes", "gemm_f16", "gemm_f16_num_tiles",
     "gemm_f16_tile_name", "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout",
     "mr_status_str", "mr_version",
 )
@@ -47,6 +48,10 @@ def _load() -> ctypes.CDLL:
     L.mrgemv_bf16_ex.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, U32, P]
     L.mrgemv_bf16_plan.argtypes = [I32, I32, I32, U32, I32, I32, P]
     L.router_topk.argtypes = [P, I64, I32, I32, I32, P, P, I64, P]
+    L.router_gemv_topk.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, P, P, I64, P,
+                                   ctypes.c_size_t, U32, P]
+    L.router_gemv_topk_workspace_bytes.argtypes = [I32, I32, I32]
+    L.router_gemv_topk_workspace_bytes.restype = ctypes.c_size_t
     L.gemm_f16.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, I32, I32, P]
     L.gemm_f16_num_tiles.argtypes = []
     L.gemm_f16_tile_name.argtypes = [I32]
@@ -58,7 +63,7 @@ def _load() -> ctypes.CDLL:
     L.mr_status_str.restype = ctypes.c_char_p
     L.mr_version.argtypes = []
     L.mr_version.restype = ctypes.c_char_p
-    for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "gemm_f16", "gemm_f16_num_tiles",
+    for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk", "gemm_f16", "gemm_f16_num_tiles",
                  "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     return L
@@ -138,6 +143,46 @@ def router_topk(logits, topk: int, idx, val=None, stream=None) -> None:
         vptr = val.data_ptr()
     st = lib.router_topk(logits.data_ptr(), ldl, m, n, topk, idx.data_ptr(), vptr, ldo, _stream(stream))
     _check(st, "router_topk")
+
+
+MR_ROUTER_TICKET_BYTES = 256
+
+
+def router_gemv_topk_workspace_bytes(m: int, n: int, logits_provided: bool) -> int:
+    return int(lib.router_gemv_topk_workspace_bytes(m, n, 1 if logits_provided else 0))
+
+
+def router_gemv_topk(A, Wt, topk: int, idx, val=None, logits=None, workspace=None, stream=None,
+                     flags: int = 0) -> None:
+    """GEMV + per-row top-k in one launch.  ``workspace``: a CUDA tensor of at
+    least router_gemv_topk_workspace_bytes(...) bytes whose first 256 bytes are
+    zero before the first call (each call leaves them zero)."""
+    m, k, lda = _rows(A, "A")
+    n, kw, ldw = _rows(Wt, "Wt")
+    if kw != k:
+        raise ValueError("A and Wt disagree on k")
+    mi, ki, ldo = _rows(idx, "idx")
+    if mi != m or ki < topk:
+        raise ValueError("idx shape mismatch")
+    lptr, ldl = None, n
+    if logits is not None:
+        ml, nl, ldl = _rows(logits, "logits")
+        if ml != m or nl != n:
+            raise ValueError("logits shape mismatch")
+        lptr = logits.data_ptr()
+    vptr = None
+    if val is not None:
+        mv, kv, ldv = _rows(val, "val")
+        if mv != m or kv < topk or ldv != ldo:
+            raise ValueError("val must match idx's shape and stride")
+        vptr = val.data_ptr()
+    if workspace is None:
+        raise ValueError("router_gemv_topk needs a zero-initialised workspace tensor")
+    wbytes = workspace.numel() * workspace.element_size()
+    st = lib.router_gemv_topk(A.data_ptr(), lda, Wt.data_ptr(), ldw, lptr, ldl, m, n, k, topk,
+                              idx.data_ptr(), vptr, ldo, workspace.data_ptr(), wbytes, flags,
+                              _stream(stream))
+    _check(st, "router_gemv_topk")
 
 
 def gemm_f16(A, Wt, C, tile_id: int = -1, in_dtype: int | None = None, stream=None) -> None:

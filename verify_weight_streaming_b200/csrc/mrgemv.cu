@@ -33,6 +33,7 @@
 //  * Every wait is an mbarrier wait bounded in time; nothing uses bar.sync
 //    after the prologue, so a wait that runs out cannot strand other warps.
 #include "common.cuh"
+#include "topk_core.cuh"
 
 #include <algorithm>
 #include <mutex>
@@ -57,6 +58,12 @@ struct Params {
     int S;          // ring slots
     uint32_t a_bytes;     // shared bytes reserved for A (MB rows)
     uint32_t slot_bytes;  // CG * k * 2
+    // Fused router (top-k of each row after the GEMV), unused otherwise.
+    int topk;
+    int32_t *idx;
+    float *val;
+    int64_t ldo;
+    uint32_t *ticket;     // CTAs that finished their columns (0 between calls)
 };
 
 // k-slice split: a function of k alone (never of m), so the reduction tree of
@@ -70,6 +77,14 @@ __host__ __device__ inline int k_warps(int k) {
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// 8-byte load from shared memory by 32-bit shared address (always LDS, never
+// a generic load).
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
 
 // Packed pairs of fp32 in one 64-bit register pair (low half first).
 __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
@@ -136,6 +151,9 @@ struct Smem {
     uint64_t *red_full;   // [CWG]
     uint64_t *red_free;   // [CWG]
     uint64_t *a_full;     // [1]
+    uint64_t *cta_done;   // [1] every warp's logits are stored (fused router)
+    uint64_t *decided;    // [1] thread 0 knows whether this CTA finished last
+    uint32_t *is_last;    // [2]
     float *red;           // [CWG][KW][32][VPL]
 };
 
@@ -153,7 +171,9 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     const uint32_t par = chunk_groups > 0 ? 0u : (uint32_t)(g / p.S) & 1u;
     if (!mbar_wait_bounded(smem_u32(&sm.full[bar_idx]), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
 
-    const uint16_t *w = reinterpret_cast<const uint16_t *>(sm.ring + (size_t)slot * p.slot_bytes);
+    const uint32_t w_s = smem_u32(sm.ring + (size_t)slot * p.slot_bytes);
+    const uint32_t a_s = smem_u32(sm.a);
+    const uint32_t row_b = (uint32_t)k * 2u;
     // acc[rp][j] holds rows (2rp, 2rp+1) of column j: one fp32 chain per
     // (row, column), over this lane's k positions in ascending order.
     constexpr int RP = MB / 2;
@@ -168,7 +188,7 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
         uint64_t wd[4][NC];  // (w, w) for element e of the chunk, column j
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
-            const uint2 raw = *reinterpret_cast<const uint2 *>(w + (size_t)j * k + 4 * q);
+            const uint2 raw = lds64(w_s + (uint32_t)j * row_b + 8u * (uint32_t)q);
             const float w0 = bf16lo(raw.x), w1 = bf16hi(raw.x), w2 = bf16lo(raw.y), w3 = bf16hi(raw.y);
             wd[0][j] = pack2(w0, w0);
             wd[1][j] = pack2(w1, w1);
@@ -177,8 +197,8 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
         }
 #pragma unroll
         for (int rp = 0; rp < RP; ++rp) {
-            const uint2 r0 = *reinterpret_cast<const uint2 *>(sm.a + (size_t)(2 * rp) * k + 4 * q);
-            const uint2 r1 = *reinterpret_cast<const uint2 *>(sm.a + (size_t)(2 * rp + 1) * k + 4 * q);
+            const uint2 r0 = lds64(a_s + (uint32_t)(2 * rp) * row_b + 8u * (uint32_t)q);
+            const uint2 r1 = lds64(a_s + (uint32_t)(2 * rp + 1) * row_b + 8u * (uint32_t)q);
             const uint64_t a0 = pack2(bf16lo(r0.x), bf16lo(r1.x));
             const uint64_t a1 = pack2(bf16hi(r0.x), bf16hi(r1.x));
             const uint64_t a2 = pack2(bf16lo(r0.y), bf16lo(r1.y));
@@ -260,7 +280,7 @@ __device__ __forceinline__ bool run_group(const Params &p, const Smem &sm, int g
     return do_group<MB, NC, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end, chunk_groups);
 }
 
-template <int MB, int CG>
+template <int MB, int CG, bool FUSED>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     constexpr int VPL = Scatter<MB * CG>::kPerLane;
@@ -284,7 +304,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     sm.red_full = sm.empty + p.S;
     sm.red_free = sm.red_full + p.CWG;
     sm.a_full = sm.red_free + p.CWG;
-    sm.red = reinterpret_cast<float *>(sm.a_full + 2);
+    sm.cta_done = sm.a_full + 1;
+    sm.decided = sm.a_full + 2;
+    sm.is_last = reinterpret_cast<uint32_t *>(sm.a_full + 3);
+    sm.red = reinterpret_cast<float *>(sm.a_full + 4);
 
     // Groups per copy chunk when no slot is refilled (0 when slots are refilled).
     const int chunk_groups = ng <= p.S ? (int)max(1u, (16384u + p.slot_bytes - 1) / p.slot_bytes) : 0;
@@ -311,6 +334,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             mbar_init(smem_u32(&sm.empty[s]), (uint32_t)p.KW);
         }
         mbar_init(smem_u32(sm.a_full), 1);
+        if constexpr (FUSED) {
+            mbar_init(smem_u32(sm.cta_done), (uint32_t)(blockDim.x / 32));
+            mbar_init(smem_u32(sm.decided), 1);
+        }
         if (p.KW > 1) {
             for (int c = 0; c < p.CWG; ++c) {
                 mbar_init(smem_u32(&sm.red_full[c]), (uint32_t)(p.KW - 1) * 32u);
@@ -364,7 +391,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
                 make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
-    if (!mbar_wait_bounded(smem_u32(sm.a_full), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
+    bool failed = !mbar_wait_bounded(smem_u32(sm.a_full), 0u, MR_DEVERR_GEMV_TIMEOUT);
 
     const int slice = warp % p.KW;
     const int cw = warp / p.KW;
@@ -373,18 +400,58 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     const int q_end = (int)(((int64_t)(slice + 1) * q_total) / p.KW);
 
     int it = 0;
-    for (int g = cw; g < ng; g += p.CWG, ++it) {
+    for (int g = cw; g < ng && !failed; g += p.CWG, ++it) {
         const int col0 = c_begin + g * CG;
         const int ncol = min(CG, c_end - col0);
-        const bool ok =
-            run_group<MB, CG, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end, chunk_groups);
-        if (!ok) return;
+        if (!run_group<MB, CG, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end, chunk_groups)) {
+            failed = true;
+            break;
+        }
         // Refill the slot with group g + S once every slice has released it.
         if (slice == 0 && lane == 0 && g + p.S < ng) {
             const int slot = g % p.S;
             const uint32_t par = (uint32_t)(g / p.S) & 1u;
-            if (!mbar_wait_bounded(smem_u32(&sm.empty[slot]), par, MR_DEVERR_GEMV_TIMEOUT)) return;
+            if (!mbar_wait_bounded(smem_u32(&sm.empty[slot]), par, MR_DEVERR_GEMV_TIMEOUT)) {
+                failed = true;
+                break;
+            }
             issue_group(g + p.S);
+        }
+    }
+
+    if constexpr (FUSED) {
+        // Router top-k in the same launch: the CTA that finishes its columns
+        // last (atomic ticket) selects the top-k of every row from the logits
+        // all CTAs stored.  Every warp arrives even after a failed wait, so
+        // thread 0's wait below ends.
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(sm.cta_done));
+        if (tid == 0) {
+            uint32_t last = 0;
+            if (mbar_wait_bounded(smem_u32(sm.cta_done), 0u, MR_DEVERR_GEMV_TIMEOUT)) {
+                __threadfence();
+                const uint32_t t = atomicAdd(p.ticket, 1u);
+                if (t == (uint32_t)p.G - 1u) {
+                    last = 1;
+                    *p.ticket = 0u;  // leave the counter at zero for the next call
+                }
+            }
+            *sm.is_last = last;
+            mbar_arrive(smem_u32(sm.decided));
+        }
+        if (!mbar_wait_bounded(smem_u32(sm.decided), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
+        if (*sm.is_last == 0u) return;
+        __threadfence();
+        const int nwarps = blockDim.x >> 5;
+        for (int r = warp; r < p.m; r += nwarps) {
+            const float *x = p.C + (int64_t)r * p.ldc;
+            const uint64_t best = topk::warp_topk_segments<4>(x, p.n, p.topk, lane, 0, 1, 0ull);
+            if (lane < p.topk) {
+                const uint32_t j = topk::key_index(best);
+                p.idx[(int64_t)r * p.ldo + lane] = (int32_t)j;
+                if (p.val) p.val[(int64_t)r * p.ldo + lane] = x[j];
+            }
         }
     }
 }
@@ -398,14 +465,17 @@ template <int MB>
 constexpr int col_group() { return MB <= 8 ? 8 : 4; }
 inline int col_group_rt(int MB) { return MB <= 8 ? 8 : 4; }
 
-KernelFn kernel_for(int MB) {
+template <bool FUSED>
+KernelFn kernel_for_mb(int MB) {
     switch (MB) {
-        case 2: return gemv_kernel<2, col_group<2>()>;
-        case 4: return gemv_kernel<4, col_group<4>()>;
-        case 8: return gemv_kernel<8, col_group<8>()>;
-        default: return gemv_kernel<16, col_group<16>()>;
+        case 2: return gemv_kernel<2, col_group<2>(), FUSED>;
+        case 4: return gemv_kernel<4, col_group<4>(), FUSED>;
+        case 8: return gemv_kernel<8, col_group<8>(), FUSED>;
+        default: return gemv_kernel<16, col_group<16>(), FUSED>;
     }
 }
+
+KernelFn kernel_for(int MB, bool fused) { return fused ? kernel_for_mb<true>(MB) : kernel_for_mb<false>(MB); }
 
 // Rows are processed in pairs, so a single row runs in the 2-row kernel with a zero second row.
 int row_bucket(int m) { return m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
@@ -418,10 +488,12 @@ cudaError_t ensure_attributes(int device) {
     if (device >= 0 && device < 64 && g_attr_done[device]) return cudaSuccess;
     const int optin = mr_host::max_smem_optin();
     const int mbs[] = {2, 4, 8, 16};
-    for (int mb : mbs) {
-        cudaError_t e = cudaFuncSetAttribute(kernel_for(mb), cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-        if (e != cudaSuccess) return e;
-    }
+    for (int mb : mbs)
+        for (int fused = 0; fused < 2; ++fused) {
+            cudaError_t e = cudaFuncSetAttribute(kernel_for(mb, fused != 0),
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+            if (e != cudaSuccess) return e;
+        }
     if (device >= 0 && device < 64) g_attr_done[device] = true;
     return cudaSuccess;
 }
@@ -458,7 +530,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     pl.a_bytes = (uint32_t)(((size_t)pl.MB * k * 2 + 127) / 128 * 128);
     pl.slot_bytes = (uint32_t)pl.CG * (uint32_t)k * 2u;
     const size_t vpl = (size_t)std::max(1, pl.MB * pl.CG / 32);
-    const size_t fixed = pl.a_bytes + 16 * (size_t)(2 * ng_max + 2 * cwg0) + 16 +
+    const size_t fixed = pl.a_bytes + 16 * (size_t)(2 * ng_max + 2 * cwg0) + 32 +
                          (size_t)cwg0 * pl.KW * 32 * vpl * 4 + 64;
     const size_t pdl_budget = 110 * 1024;
     const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, (size_t)optin) : (size_t)optin;
@@ -482,7 +554,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
         pl.CWG = std::max(1, std::min(cwg0, s_max / 2));
         pl.S = (s_max / pl.CWG) * pl.CWG;
     }
-    pl.smem = pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 16 * (size_t)(pl.S + pl.CWG) + 16 +
+    pl.smem = pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 16 * (size_t)(pl.S + pl.CWG) + 32 +
               (size_t)pl.CWG * pl.KW * 32 * vpl * 4;
     if (pl.smem > (size_t)optin) return MR_ERR_UNSUPPORTED;
     return MR_OK;
@@ -509,10 +581,20 @@ extern "C" mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t 
     return MR_OK;
 }
 
-extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw,
-                                    float *C, int64_t ldc, int32_t m, int32_t n, int32_t k,
-                                    uint32_t flags, void *stream) {
-    using namespace mr::gemv;
+namespace mr {
+namespace gemv {
+
+struct FusedArgs {
+    int topk;
+    int32_t *idx;
+    float *val;
+    int64_t ldo;
+    uint32_t *ticket;
+};
+
+// Validate, plan and launch; `fused` adds the router top-k of every row.
+mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *C, int64_t ldc, int32_t m,
+                 int32_t n, int32_t k, uint32_t flags, void *stream, const FusedArgs *fused) {
     if (!A || !Wt || !C) return MR_ERR_INVALID_ARG;
     if (m < 1 || n < 1 || k < 1) return MR_ERR_INVALID_ARG;
     if (lda < k || ldw < k || ldc < n) return MR_ERR_INVALID_ARG;
@@ -531,7 +613,7 @@ extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, 
     const mr_status st = make_plan(m, n, k, flags, sms, optin, pl);
     if (st != MR_OK) return st;
 
-    Params p;
+    Params p = {};
     p.A = static_cast<const uint16_t *>(A);
     p.lda = lda;
     p.Wt = static_cast<const uint16_t *>(Wt);
@@ -547,6 +629,13 @@ extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, 
     p.S = pl.S;
     p.a_bytes = pl.a_bytes;
     p.slot_bytes = pl.slot_bytes;
+    if (fused) {
+        p.topk = fused->topk;
+        p.idx = fused->idx;
+        p.val = fused->val;
+        p.ldo = fused->ldo;
+        p.ticket = fused->ticket;
+    }
 
     e = ensure_attributes(device);
     if (e != cudaSuccess) return mr_host::cuda_status(e);
@@ -561,8 +650,41 @@ extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = (flags & MR_GEMV_PDL) ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kernel_for(pl.MB), p);
+    e = cudaLaunchKernelEx(&cfg, kernel_for(pl.MB, fused != nullptr), p);
     return mr_host::cuda_status(e);
+}
+
+}  // namespace gemv
+}  // namespace mr
+
+extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw,
+                                    float *C, int64_t ldc, int32_t m, int32_t n, int32_t k,
+                                    uint32_t flags, void *stream) {
+    return mr::gemv::launch(A, lda, Wt, ldw, C, ldc, m, n, k, flags, stream, nullptr);
+}
+
+extern "C" size_t router_gemv_topk_workspace_bytes(int32_t m, int32_t n, int32_t logits_provided) {
+    if (m < 1 || n < 1) return 0;
+    return MR_ROUTER_TICKET_BYTES + (logits_provided ? 0 : (size_t)m * (size_t)n * sizeof(float));
+}
+
+extern "C" mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *logits,
+                                      int64_t ldl, int32_t m, int32_t n, int32_t k, int32_t topk, int32_t *idx,
+                                      float *val, int64_t ldo, void *workspace, size_t workspace_bytes,
+                                      uint32_t flags, void *stream) {
+    if (!idx || !workspace) return MR_ERR_INVALID_ARG;
+    if (m < 1 || n < 1 || topk < 1 || topk > n || ldo < topk) return MR_ERR_INVALID_ARG;
+    if (topk > 32) return MR_ERR_UNSUPPORTED;
+    if (((uintptr_t)workspace & 255u) || ((uintptr_t)idx & 3u) || ((uintptr_t)val & 3u)) return MR_ERR_MISALIGNED;
+    if (workspace_bytes < router_gemv_topk_workspace_bytes(m, n, logits != nullptr)) return MR_ERR_INVALID_ARG;
+    float *C = logits;
+    int64_t ldc = ldl;
+    if (!C) {
+        C = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + MR_ROUTER_TICKET_BYTES);
+        ldc = n;
+    }
+    mr::gemv::FusedArgs fa = {topk, idx, val, ldo, static_cast<uint32_t *>(workspace)};
+    return mr::gemv::launch(A, lda, Wt, ldw, C, ldc, m, n, k, flags, stream, &fa);
 }
 
 extern "C" mr_status mrgemv_bf16(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *C,

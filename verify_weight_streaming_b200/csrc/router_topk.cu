@@ -16,58 +16,14 @@
 // selected indices so they match bit for bit (a -0.0 stays -0.0).
 #include "common.cuh"
 
+#include "topk_core.cuh"
+
 namespace mr {
 namespace topk {
 
 constexpr int kWarps = 4;
 constexpr int kP = 4;              // elements per lane per segment
-constexpr int kSeg = 32 * kP;      // elements per warp segment
 constexpr int kMaxK = 32;
-
-__device__ __forceinline__ uint64_t make_key(float v, uint32_t idx) {
-    uint32_t b = __float_as_uint(v);
-    uint32_t hi;
-    if (v != v) {
-        hi = 0xFFFFFFFFu;
-    } else {
-        if ((b & 0x7FFFFFFFu) == 0u) b = 0u;
-        hi = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    }
-    return ((uint64_t)hi << 32) | (uint64_t)(0xFFFFFFFFu - idx);
-}
-
-// Sort L keys descending (insertion network, compile-time indices).
-template <int L>
-__device__ __forceinline__ void sort_desc(uint64_t (&x)[L]) {
-#pragma unroll
-    for (int i = 1; i < L; ++i)
-#pragma unroll
-        for (int j = i; j > 0; --j) {
-            const uint64_t a = x[j - 1], b = x[j];
-            const bool sw = b > a;
-            x[j - 1] = sw ? b : a;
-            x[j] = sw ? a : b;
-        }
-}
-
-// K rounds of warp-wide maximum over the lanes' heads (each lane's keys sorted
-// descending).  Lane t receives the t-th largest key (0 if fewer exist).
-template <int L>
-__device__ __forceinline__ uint64_t warp_select(uint64_t (&x)[L], int K, int lane) {
-    uint64_t mine = 0;
-#pragma unroll 1
-    for (int t = 0; t < K; ++t) {
-        const uint32_t hi = (uint32_t)(x[0] >> 32), lo = (uint32_t)x[0];
-        const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
-        const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
-        const bool win = (hi == mhi) && (lo == mlo);
-#pragma unroll
-        for (int i = 0; i < L - 1; ++i) x[i] = win ? x[i + 1] : x[i];
-        if (win) x[L - 1] = 0;
-        if (lane == t) mine = ((uint64_t)mhi << 32) | mlo;
-    }
-    return mine;
-}
 
 __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float *__restrict__ logits, int64_t ldl,
                                                           int n, int K, int32_t *__restrict__ idx,
@@ -77,19 +33,7 @@ __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float *__restri
     const int64_t row = blockIdx.x;
     const float *x = logits + row * ldl;
 
-    uint64_t run = 0;
-    for (int seg = warp; (int64_t)seg * kSeg < n; seg += kWarps) {
-        const int base = seg * kSeg;
-        uint64_t keys[kP + 1];
-#pragma unroll
-        for (int i = 0; i < kP; ++i) {
-            const int j = base + lane + 32 * i;
-            keys[i] = j < n ? make_key(x[j], (uint32_t)j) : 0ull;
-        }
-        keys[kP] = run;
-        sort_desc(keys);
-        run = warp_select(keys, K, lane);
-    }
+    const uint64_t run = warp_topk_segments<kP>(x, n, K, lane, warp, kWarps, 0ull);
     cand[warp][lane] = lane < K ? run : 0ull;
     __syncthreads();
     if (warp == 0) {
@@ -99,7 +43,7 @@ __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float *__restri
         sort_desc(keys);
         const uint64_t best = warp_select(keys, K, lane);
         if (lane < K) {
-            const uint32_t j = 0xFFFFFFFFu - (uint32_t)best;
+            const uint32_t j = key_index(best);
             idx[row * ldo + lane] = (int32_t)j;
             if (val) val[row * ldo + lane] = x[j];
         }

@@ -1,0 +1,86 @@
+// Warp-level top-k under the total order of the router selection: value
+// descending, equal values by index ascending, -0.0 equal to +0.0, any NaN
+// above +inf.  Shared by router_topk and the fused router kernel.
+#pragma once
+
+#include <stdint.h>
+
+namespace mr {
+namespace topk {
+
+// 64-bit key whose unsigned order is the total order: the high word maps the
+// float to an unsigned integer increasing with its value (sign-magnitude
+// flip, -0.0 folded onto +0.0, every NaN mapped to the maximum); the low word
+// is 0xFFFFFFFF - index, so the lower index of two equal values has the
+// larger key.  0 is never a key (it would need index 0xFFFFFFFF) and marks an
+// empty entry.
+__device__ __forceinline__ uint64_t make_key(float v, uint32_t idx) {
+    uint32_t b = __float_as_uint(v);
+    uint32_t hi;
+    if (v != v) {
+        hi = 0xFFFFFFFFu;
+    } else {
+        if ((b & 0x7FFFFFFFu) == 0u) b = 0u;
+        hi = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    }
+    return ((uint64_t)hi << 32) | (uint64_t)(0xFFFFFFFFu - idx);
+}
+
+__device__ __forceinline__ uint32_t key_index(uint64_t key) { return 0xFFFFFFFFu - (uint32_t)key; }
+
+// Sort L keys descending (insertion network, compile-time indices).
+template <int L>
+__device__ __forceinline__ void sort_desc(uint64_t (&x)[L]) {
+#pragma unroll
+    for (int i = 1; i < L; ++i)
+#pragma unroll
+        for (int j = i; j > 0; --j) {
+            const uint64_t a = x[j - 1], b = x[j];
+            const bool sw = b > a;
+            x[j - 1] = sw ? b : a;
+            x[j] = sw ? a : b;
+        }
+}
+
+// K rounds of warp-wide maximum over the lanes' heads (each lane's keys
+// sorted descending).  Lane t receives the t-th largest key (0 if fewer exist).
+template <int L>
+__device__ __forceinline__ uint64_t warp_select(uint64_t (&x)[L], int K, int lane) {
+    uint64_t mine = 0;
+#pragma unroll 1
+    for (int t = 0; t < K; ++t) {
+        const uint32_t hi = (uint32_t)(x[0] >> 32), lo = (uint32_t)x[0];
+        const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+        const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+        const bool win = (hi == mhi) && (lo == mlo);
+#pragma unroll
+        for (int i = 0; i < L - 1; ++i) x[i] = win ? x[i + 1] : x[i];
+        if (win) x[L - 1] = 0;
+        if (lane == t) mine = ((uint64_t)mhi << 32) | mlo;
+    }
+    return mine;
+}
+
+// Running top-K of elements [begin, end) of a row taken by one warp in
+// segments of 32*P elements starting at `begin` and stepping `stride`
+// segments; `run` is the warp's running list (lane t holds rank t).
+template <int P>
+__device__ __forceinline__ uint64_t warp_topk_segments(const float *x, int n, int K, int lane, int seg0,
+                                                       int seg_stride, uint64_t run) {
+    for (int seg = seg0; (int64_t)seg * 32 * P < n; seg += seg_stride) {
+        const int base = seg * 32 * P;
+        uint64_t keys[P + 1];
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            const int j = base + lane + 32 * i;
+            keys[i] = j < n ? make_key(x[j], (uint32_t)j) : 0ull;
+        }
+        keys[P] = run;
+        sort_desc(keys);
+        run = warp_select(keys, K, lane);
+    }
+    return run;
+}
+
+}  // namespace topk
+}  // namespace mr
