@@ -138,6 +138,34 @@ mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt, int64_t l
 size_t router_gemv_topk_workspace_bytes(int32_t m, int32_t n, int32_t logits_provided);
 
 /*
+ * router_gemv_topk_noalloc -- router_gemv_topk without a workspace argument,
+ * for callers that cannot allocate device memory (a host whose device memory
+ * all belongs to its own pool and accounting, a plug-in that may not call
+ * cudaMalloc) and so cannot hand in a workspace.  The pages have no
+ * counterpart: this is a convenience of this library.
+ *
+ * Arguments and outputs are those of router_gemv_topk.  The scratch it needs
+ * (the ticket block, and the logits when `logits` is NULL) is a fixed 256 KiB
+ * device array inside the library, held by every GPU that loads the library
+ * until the process exits.  With logits == NULL, m * n may not exceed
+ * router_gemv_topk_noalloc_max_logits() (65472 values, e.g. 16 x 4092);
+ * larger sizes are rejected with MR_ERR_UNSUPPORTED before anything runs.
+ * The call allocates nothing: its first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current, so make
+ * that first call before any stream capture.  Each call clears the ticket on
+ * `stream` (cudaMemsetAsync) and then launches.  Every call shares the one
+ * array, so calls that overlap on the GPU (other streams, or overlapping
+ * launches) race and must not be issued.
+ */
+mr_status router_gemv_topk_noalloc(const void *A, int64_t lda, const void *Wt, int64_t ldw,
+                                   float *logits, int64_t ldl, int32_t m, int32_t n, int32_t k,
+                                   int32_t topk, int32_t *idx, float *val, int64_t ldo,
+                                   uint32_t flags, void *stream);
+
+/* Largest m * n router_gemv_topk_noalloc accepts when logits is NULL. */
+size_t router_gemv_topk_noalloc_max_logits(void);
+
+/*
  * router_topk -- per-row top-k of fp32 logits, one CTA per row.
  *
  * The multi-row top-10 launch of Strata PR #109 ("What", router bullet: the

@@ -21,7 +21,7 @@ MR_DEVERR_GEMV_TIMEOUT, MR_DEVERR_GEMM_TIMEOUT, MR_DEVERR_TOPK_TIMEOUT, MR_DEVER
 
 EXPORTS = (
     "mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
-    "router_gemv_topk_workspace_bytes", "gemm_f16", "gemm_f16_num_tiles",
+    "router_gemv_topk_workspace_bytes", "router_gemv_topk_noalloc", "router_gemv_topk_noalloc_max_logits", "gemm_f16", "gemm_f16_num_tiles",
     "gemm_f16_tile_name", "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout",
     "mr_status_str", "mr_version",
 )
@@ -52,6 +52,9 @@ def _load() -> ctypes.CDLL:
                                    ctypes.c_size_t, U32, P]
     L.router_gemv_topk_workspace_bytes.argtypes = [I32, I32, I32]
     L.router_gemv_topk_workspace_bytes.restype = ctypes.c_size_t
+    L.router_gemv_topk_noalloc.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, P, P, I64, U32, P]
+    L.router_gemv_topk_noalloc_max_logits.argtypes = []
+    L.router_gemv_topk_noalloc_max_logits.restype = ctypes.c_size_t
     L.gemm_f16.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, I32, I32, P]
     L.gemm_f16_num_tiles.argtypes = []
     L.gemm_f16_tile_name.argtypes = [I32]
@@ -63,7 +66,8 @@ def _load() -> ctypes.CDLL:
     L.mr_status_str.restype = ctypes.c_char_p
     L.mr_version.argtypes = []
     L.mr_version.restype = ctypes.c_char_p
-    for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk", "gemm_f16", "gemm_f16_num_tiles",
+    for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
+                 "router_gemv_topk_noalloc", "gemm_f16", "gemm_f16_num_tiles",
                  "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     return L

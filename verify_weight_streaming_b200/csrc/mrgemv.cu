@@ -92,15 +92,8 @@ __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
     return r;
 }
-__device__ __forceinline__ float lo_of(uint64_t v) {
-    float lo, hi;
+__device__ __forceinline__ void unpack2(uint64_t v, float &lo, float &hi) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return lo;
-}
-__device__ __forceinline__ float hi_of(uint64_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return hi;
 }
 
 // acc.lo = fma(a.lo, b.lo, acc.lo); acc.hi = fma(a.hi, b.hi, acc.hi): two
@@ -222,8 +215,7 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     for (int rp = 0; rp < RP; ++rp)
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
-            v[(2 * rp) * NC + j] = lo_of(acc[rp][j]);
-            v[(2 * rp + 1) * NC + j] = hi_of(acc[rp][j]);
+            unpack2(acc[rp][j], v[(2 * rp) * NC + j], v[(2 * rp + 1) * NC + j]);
         }
     int base = 0;
     ReduceScatter<V, 16>::run(v, lane, base);
@@ -690,4 +682,62 @@ extern "C" mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt
 extern "C" mr_status mrgemv_bf16(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *C,
                                  int64_t ldc, int32_t m, int32_t n, int32_t k, void *stream) {
     return mrgemv_bf16_ex(A, lda, Wt, ldw, C, ldc, m, n, k, 0u, stream);
+}
+
+// ---------------------------------------------------------------------------
+// router_gemv_topk_noalloc: router_gemv_topk for callers that cannot provide a
+// workspace because they cannot allocate device memory -- for example a host
+// whose device memory is all owned by its own pool and accounting, or a
+// plug-in that is not allowed to call cudaMalloc.  The scratch (ticket block,
+// then the logits when the caller passes none) is one file-scope device array
+// of fixed size that every GPU loading this library holds until the process
+// exits.
+// ---------------------------------------------------------------------------
+
+namespace mr {
+namespace gemv {
+
+constexpr size_t kNoAllocScratchBytes = 256u * 1024u;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mutex;
+void *g_scratch_ptr[64] = {};
+
+// The array's device address, looked up once per device with that device
+// current.  (In host code `g_noalloc_scratch` names a host-side stand-in, not
+// device memory, so it must never be passed to a kernel directly.)
+mr_status noalloc_scratch(void **out) {
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= 64) return MR_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[device]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MR_ERR_CUDA;
+        g_scratch_ptr[device] = ptr;
+    }
+    *out = g_scratch_ptr[device];
+    return MR_OK;
+}
+
+}  // namespace gemv
+}  // namespace mr
+
+extern "C" size_t router_gemv_topk_noalloc_max_logits(void) {
+    return (mr::gemv::kNoAllocScratchBytes - MR_ROUTER_TICKET_BYTES) / sizeof(float);
+}
+
+extern "C" mr_status router_gemv_topk_noalloc(const void *A, int64_t lda, const void *Wt, int64_t ldw,
+                                              float *logits, int64_t ldl, int32_t m, int32_t n, int32_t k,
+                                              int32_t topk, int32_t *idx, float *val, int64_t ldo, uint32_t flags,
+                                              void *stream) {
+    if (m < 1 || n < 1) return MR_ERR_INVALID_ARG;
+    if (!logits && (size_t)m * (size_t)n > router_gemv_topk_noalloc_max_logits()) return MR_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    const mr_status st = mr::gemv::noalloc_scratch(&scratch);
+    if (st != MR_OK) return st;
+    // The array keeps whatever the last call left; the ticket must start at zero.
+    if (cudaMemsetAsync(scratch, 0, MR_ROUTER_TICKET_BYTES, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return MR_ERR_CUDA;
+    return router_gemv_topk(A, lda, Wt, ldw, logits, ldl, m, n, k, topk, idx, val, ldo, scratch,
+                            mr::gemv::kNoAllocScratchBytes, flags, stream);
 }
