@@ -436,9 +436,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
         if (*sm.is_last == 0u) return;
         __threadfence();
         const int nwarps = blockDim.x >> 5;
+        uint64_t *tk = reinterpret_cast<uint64_t *>(sm.red + (size_t)p.CWG * p.KW * 32 * VPL) + warp * 64;
         for (int r = warp; r < p.m; r += nwarps) {
             const float *x = p.C + (int64_t)r * p.ldc;
-            const uint64_t best = topk::warp_topk_segments<4>(x, p.n, p.topk, lane, 0, 1, 0ull);
+            const uint64_t best = topk::warp_topk_fast<16>(x, p.n, p.topk, lane, 0, 1, 0ull, tk);
             if (lane < p.topk) {
                 const uint32_t j = topk::key_index(best);
                 p.idx[(int64_t)r * p.ldo + lane] = (int32_t)j;
@@ -508,7 +509,7 @@ struct Plan {
 // CWG so that slot s is only ever consumed by column warp s % CWG, which waits
 // for the slot's uses strictly in order (a parity wait is then never more
 // than one phase ahead of the barrier).
-mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Plan &pl) {
+mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Plan &pl, bool fused = false) {
     if (m < 1 || n < 1 || k < 8 || sms < 1 || optin < 1) return MR_ERR_INVALID_ARG;
     if (k % 8 != 0) return MR_ERR_MISALIGNED;
     if (m > kMaxRows) return MR_ERR_UNSUPPORTED;
@@ -522,7 +523,8 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     pl.a_bytes = (uint32_t)(((size_t)pl.MB * k * 2 + 127) / 128 * 128);
     pl.slot_bytes = (uint32_t)pl.CG * (uint32_t)k * 2u;
     const size_t vpl = (size_t)std::max(1, pl.MB * pl.CG / 32);
-    const size_t fixed = pl.a_bytes + 16 * (size_t)(2 * ng_max + 2 * cwg0) + 32 +
+    const size_t topk_bytes = fused ? (size_t)kMaxWarps * 64 * 8 : 0;
+    const size_t fixed = topk_bytes + pl.a_bytes + 16 * (size_t)(2 * ng_max + 2 * cwg0) + 32 +
                          (size_t)cwg0 * pl.KW * 32 * vpl * 4 + 64;
     const size_t pdl_budget = 110 * 1024;
     const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, (size_t)optin) : (size_t)optin;
@@ -546,7 +548,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
         pl.CWG = std::max(1, std::min(cwg0, s_max / 2));
         pl.S = (s_max / pl.CWG) * pl.CWG;
     }
-    pl.smem = pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 16 * (size_t)(pl.S + pl.CWG) + 32 +
+    pl.smem = topk_bytes + pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 16 * (size_t)(pl.S + pl.CWG) + 32 +
               (size_t)pl.CWG * pl.KW * 32 * vpl * 4;
     if (pl.smem > (size_t)optin) return MR_ERR_UNSUPPORTED;
     return MR_OK;
@@ -602,7 +604,7 @@ mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float 
     const int optin = mr_host::max_smem_optin();
     if (sms <= 0 || optin <= 0) return MR_ERR_CUDA;
     Plan pl;
-    const mr_status st = make_plan(m, n, k, flags, sms, optin, pl);
+    const mr_status st = make_plan(m, n, k, flags, sms, optin, pl, fused != nullptr);
     if (st != MR_OK) return st;
 
     Params p = {};

@@ -9,11 +9,13 @@
 // folded onto +0.0, every NaN mapped to the maximum); the low word is
 // 0xFFFFFFFF - index, so among equal values the lower index has the larger
 // key.  Keys are unique, and "top-k by the total order" is "the k largest
-// keys".  Each warp keeps a running top-k spread one entry per lane; every
-// segment of 32*P elements is merged into it with k rounds of a warp-wide
-// maximum (two __reduce_max_sync on the key's halves).  The CTA's warps are
-// merged the same way at the end.  Values are re-read from the logits at the
-// selected indices so they match bit for bit (a -0.0 stays -0.0).
+// keys".  Each warp keeps a running top-k spread one entry per lane and
+// merges every chunk of 32*P elements into it: a threshold from the lane
+// maxima keeps at most 32 candidates, which are ranked with shuffles in one
+// pass (k rounds of a warp-wide maximum when ties leave more than 32).  The
+// CTA's warps are merged the same way at the end.  Values are re-read from
+// the logits at the selected indices so they match bit for bit (a -0.0 stays
+// -0.0).
 #include "common.cuh"
 
 #include "topk_core.cuh"
@@ -22,26 +24,26 @@ namespace mr {
 namespace topk {
 
 constexpr int kWarps = 4;
-constexpr int kP = 4;              // elements per lane per segment
+constexpr int kP = 4;              // elements per lane per chunk (128 per warp)
 constexpr int kMaxK = 32;
 
 __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float *__restrict__ logits, int64_t ldl,
                                                           int n, int K, int32_t *__restrict__ idx,
                                                           float *__restrict__ val, int64_t ldo) {
     __shared__ uint64_t cand[kWarps][32];
+    __shared__ uint64_t scratch[kWarps][64];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row = blockIdx.x;
     const float *x = logits + row * ldl;
 
-    const uint64_t run = warp_topk_segments<kP>(x, n, K, lane, warp, kWarps, 0ull);
+    const uint64_t run = warp_topk_fast<kP>(x, n, K, lane, warp, kWarps, 0ull, scratch[warp]);
     cand[warp][lane] = lane < K ? run : 0ull;
     __syncthreads();
     if (warp == 0) {
         uint64_t keys[kWarps];
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) keys[w] = cand[w][lane];
-        sort_desc(keys);
-        const uint64_t best = warp_select(keys, K, lane);
+        const uint64_t best = warp_topk_merge<kWarps>(keys, 0ull, K, lane, scratch[0]);
         if (lane < K) {
             const uint32_t j = key_index(best);
             idx[row * ldo + lane] = (int32_t)j;

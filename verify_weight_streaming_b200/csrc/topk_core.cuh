@@ -82,5 +82,97 @@ __device__ __forceinline__ uint64_t warp_topk_segments(const float *x, int n, in
     return run;
 }
 
+// Rank of `key` among the 32 lanes' keys: how many lanes hold a larger key.
+// Keys are unique, so nonzero keys get distinct ranks.
+__device__ __forceinline__ int warp_rank(uint64_t key, int lane) {
+    int r = 0;
+#pragma unroll
+    for (int s = 1; s < 32; ++s) {
+        const uint64_t o = __shfl_sync(0xffffffffu, key, (lane + s) & 31);
+        r += o > key ? 1 : 0;
+    }
+    return r;
+}
+
+// Top-K (K <= 32) of one chunk of up to 32*P keys held P per lane, merged
+// with a running list `run` (lane t holds rank t, 0 = empty).  Fast path:
+// tau = the K-th largest lane maximum (every one of the top K keys is >= tau,
+// because the K lanes with the largest maxima each hold a key >= tau); the
+// keys >= tau are gathered through `scratch` (64 keys of shared memory per
+// warp) and, when there are at most 32, ranked with shuffles in one pass.
+// Otherwise (heavy ties) it falls back to K rounds of warp-wide maximum.
+// Returns the new running list (lane t holds rank t).
+template <int P>
+__device__ __forceinline__ uint64_t warp_topk_merge(uint64_t (&key)[P], uint64_t run, int K, int lane,
+                                                    uint64_t *scratch) {
+    uint64_t mx = run;
+#pragma unroll
+    for (int i = 0; i < P; ++i) mx = key[i] > mx ? key[i] : mx;
+    const int r0 = warp_rank(mx, lane);
+    const unsigned who = __ballot_sync(0xffffffffu, r0 == K - 1 && mx != 0ull);
+    // Fewer than K nonzero lane maxima: every nonzero key is a candidate.
+    const uint64_t tau = who ? __shfl_sync(0xffffffffu, mx, __ffs(who) - 1) : 1ull;
+    int c = (run >= tau && run != 0ull) ? 1 : 0;
+#pragma unroll
+    for (int i = 0; i < P; ++i) c += (key[i] >= tau && key[i] != 0ull) ? 1 : 0;
+    int pos = c;  // inclusive prefix sum of the counts over lanes
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, pos, d);
+        if (lane >= d) pos += o;
+    }
+    const int total = __shfl_sync(0xffffffffu, pos, 31);
+    if (total <= 32) {
+        pos -= c;
+        if (c) {
+            if (run >= tau && run != 0ull) scratch[pos++] = run;
+#pragma unroll
+            for (int i = 0; i < P; ++i)
+                if (key[i] >= tau && key[i] != 0ull) scratch[pos++] = key[i];
+        }
+        scratch[32 + lane] = 0ull;
+        __syncwarp();
+        const uint64_t cand = lane < total ? scratch[lane] : 0ull;
+        const int r = warp_rank(cand, lane);
+        __syncwarp();
+        if (cand != 0ull && r < K) scratch[32 + r] = cand;
+        __syncwarp();
+        const uint64_t out = lane < K ? scratch[32 + lane] : 0ull;
+        __syncwarp();
+        return out;
+    }
+    // Slow path: sort each lane's keys and take K rounds of the warp maximum.
+    uint64_t all[P + 1];
+#pragma unroll
+    for (int i = 0; i < P; ++i) all[i] = key[i];
+    all[P] = run;
+    sort_desc(all);
+    return warp_select(all, K, lane);
+}
+
+// Running top-K of x[0, n) taken by one warp in chunks of 32*P elements
+// (chunks seg0, seg0 + seg_stride, ...), merged into `run`.
+template <int P>
+__device__ __forceinline__ uint64_t warp_topk_fast(const float *x, int n, int K, int lane, int seg0,
+                                                   int seg_stride, uint64_t run, uint64_t *scratch) {
+    for (int seg = seg0; (int64_t)seg * 32 * P < n; seg += seg_stride) {
+        const int base = seg * 32 * P;
+        float v[P];
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            const int j = base + lane + 32 * i;
+            v[i] = j < n ? x[j] : 0.0f;
+        }
+        uint64_t keys[P];
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            const int j = base + lane + 32 * i;
+            keys[i] = j < n ? make_key(v[i], (uint32_t)j) : 0ull;
+        }
+        run = warp_topk_merge<P>(keys, run, K, lane, scratch);
+    }
+    return run;
+}
+
 }  // namespace topk
 }  // namespace mr
