@@ -661,6 +661,21 @@ def profile_case(case: str):
         C = torch.empty((m, n), dtype=torch.float32, device="cuda")
         for i in range(3):
             mr.mrgemv_bf16(A[:m], W[i], C)
+    elif case == "router_fused":
+        a16, w16 = synth.router(16)
+        pool = [torch.from_numpy(w16.view(np.int16)).cuda() for _ in range(110)]
+        A = torch.from_numpy(a16.view(np.int16)).cuda()
+        ws = torch.zeros(mr.router_gemv_topk_workspace_bytes(16, N_ROUTER, False) // 4 + 1,
+                         dtype=torch.int32, device="cuda")
+        for m in (1, 16):
+            C = torch.empty((m, N_ROUTER), dtype=torch.float32, device="cuda")
+            idx = torch.empty((m, TOPK), dtype=torch.int32, device="cuda")
+            val = torch.empty((m, TOPK), dtype=torch.float32, device="cuda")
+            for i in range(3):
+                mr.mrgemv_bf16(A[:m], pool[(3 * i + m) % len(pool)], C)
+                mr.router_topk(C, TOPK, idx, val)
+            for i in range(3):
+                mr.router_gemv_topk(A[:m], pool[(5 * i + m + 40) % len(pool)], TOPK, idx, val, workspace=ws)
     elif case == "topk":
         x = torch.randn(16, 512, device="cuda")
         idx = torch.empty((16, TOPK), dtype=torch.int32, device="cuda")

@@ -414,16 +414,19 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     if constexpr (FUSED) {
         // Router top-k in the same launch: the CTA that finishes its columns
         // last (atomic ticket) selects the top-k of every row from the logits
-        // all CTAs stored.  Every warp arrives even after a failed wait, so
-        // thread 0's wait below ends.
-        __threadfence();
+        // all CTAs stored.  Ordering: each warp's stores -> __syncwarp ->
+        // release arrive on cta_done (CTA scope) -> thread 0's acquire wait ->
+        // one acq_rel atomic at GPU scope, whose release covers what thread 0
+        // has observed; the last CTA's atomic acquires every other CTA's
+        // release, and hands it to its warps through the `decided` barrier.
+        // Every warp arrives even after a failed wait, so thread 0's wait ends.
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(sm.cta_done));
         if (tid == 0) {
             uint32_t last = 0;
             if (mbar_wait_bounded(smem_u32(sm.cta_done), 0u, MR_DEVERR_GEMV_TIMEOUT)) {
-                __threadfence();
-                const uint32_t t = atomicAdd(p.ticket, 1u);
+                uint32_t t;
+                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.ticket) : "memory");
                 if (t == (uint32_t)p.G - 1u) {
                     last = 1;
                     *p.ticket = 0u;  // leave the counter at zero for the next call
@@ -434,7 +437,6 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
         }
         if (!mbar_wait_bounded(smem_u32(sm.decided), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
         if (*sm.is_last == 0u) return;
-        __threadfence();
         const int nwarps = blockDim.x >> 5;
         uint64_t *tk = reinterpret_cast<uint64_t *>(sm.red + (size_t)p.CWG * p.KW * 32 * VPL) + warp * 64;
         for (int r = warp; r < p.m; r += nwarps) {

@@ -35,6 +35,11 @@ __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float *__restri
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row = blockIdx.x;
     const float *x = logits + row * ldl;
+    // Launched with programmatic stream serialization: let the next kernel
+    // start its prologue, and read the logits only once the kernel that
+    // produced them has completed.
+    grid_launch_dependents();
+    grid_dependency_wait();
 
     const uint64_t run = warp_topk_fast<kP>(x, n, K, lane, warp, kWarps, 0ull, scratch[warp]);
     cand[warp][lane] = lane < K ? run : 0ull;
@@ -66,6 +71,12 @@ extern "C" mr_status router_topk(const float *logits, int64_t ldl, int32_t m, in
     cfg.gridDim = dim3((unsigned)m);
     cfg.blockDim = dim3(mr::topk::kWarps * 32);
     cfg.stream = static_cast<cudaStream_t>(stream);
+    // Safe for any predecessor: the kernel waits for it before reading input.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     return mr_host::cuda_status(
         cudaLaunchKernelEx(&cfg, mr::topk::topk_kernel, logits, ldl, (int)n, (int)topk, idx, val, ldo));
 }
