@@ -208,28 +208,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // Warps 0 and 1 run their loops as whole warps (every lane waits on the
+    // same barrier) and let lane 0 issue: a lone lane spinning in try_wait
+    // beside warp-mates parked elsewhere can stall for the suspend limit.
     if (warp == 0) {
-        if (lane == 0) {
-            // Producer: stage s is reused after the MMAs reading it complete.
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t par = ((uint32_t)(kb / STAGES) & 1u) ^ 1u;
-                if (!mbar_wait_bounded(smem_u32(&empty[s]), par, MR_DEVERR_GEMM_TIMEOUT)) break;
+        // Producer: stage s is reused after the MMAs reading it complete.
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t par = ((uint32_t)(kb / STAGES) & 1u) ^ 1u;
+            if (!mbar_wait_bounded(smem_u32(&empty[s]), par, MR_DEVERR_GEMM_TIMEOUT)) break;
+            if (lane == 0) {
                 const uint32_t fb = smem_u32(&full[s]);
                 mbar_arrive_expect_tx(fb, kABytes + kBBytes);
                 tma_load_2d(sA + s * kABytes, &tmA, kb * BK, m0, fb);
                 tma_load_2d(sB + s * kBBytes, &tmB, kb * BK, n0, fb);
             }
+            __syncwarp();
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            bool ok = true;
-            for (int kb = 0; kb < nkb && ok; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t par = (uint32_t)(kb / STAGES) & 1u;
-                ok = mbar_wait_bounded(smem_u32(&full[s]), par, MR_DEVERR_GEMM_TIMEOUT);
-                if (!ok) break;
-                tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t par = (uint32_t)(kb / STAGES) & 1u;
+            ok = mbar_wait_bounded(smem_u32(&full[s]), par, MR_DEVERR_GEMM_TIMEOUT);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
                     const uint64_t ad = sw128_desc(sA + s * kABytes + kk * 32);
@@ -238,8 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(smem_u32(&empty[s]));
             }
-            if (ok) mma_commit(smem_u32(tmem_full));
+            __syncwarp();
         }
+        if (ok && lane == 0) mma_commit(smem_u32(tmem_full));
+        __syncwarp();
     } else {
         // Epilogue warps 2..5: warp w reads tensor-memory lanes 32*(w%4) .. +31.
         const int q = warp & 3;

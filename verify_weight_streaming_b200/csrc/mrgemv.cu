@@ -400,14 +400,18 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             break;
         }
         // Refill the slot with group g + S once every slice has released it.
-        if (slice == 0 && lane == 0 && g + p.S < ng) {
+        // The whole warp waits (a lone lane in try_wait beside warp-mates
+        // suspended on another barrier can stall for the suspend time limit);
+        // lane 0 then issues the copies.
+        if (slice == 0 && g + p.S < ng) {
             const int slot = g % p.S;
             const uint32_t par = (uint32_t)(g / p.S) & 1u;
             if (!mbar_wait_bounded(smem_u32(&sm.empty[slot]), par, MR_DEVERR_GEMV_TIMEOUT)) {
                 failed = true;
                 break;
             }
-            issue_group(g + p.S);
+            if (lane == 0) issue_group(g + p.S);
+            __syncwarp();
         }
     }
 
@@ -422,21 +426,31 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
         // Every warp arrives even after a failed wait, so thread 0's wait ends.
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(sm.cta_done));
-        if (tid == 0) {
-            uint32_t last = 0;
+        uint32_t last = 0;
+        if (warp == 0) {
+            // Warp 0 decides as a whole (its lanes never wait on different
+            // barriers); lane 0 takes the ticket.
             if (mbar_wait_bounded(smem_u32(sm.cta_done), 0u, MR_DEVERR_GEMV_TIMEOUT)) {
-                uint32_t t;
-                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.ticket) : "memory");
-                if (t == (uint32_t)p.G - 1u) {
-                    last = 1;
-                    *p.ticket = 0u;  // leave the counter at zero for the next call
+                if (lane == 0) {
+                    uint32_t t;
+                    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.ticket) : "memory");
+                    if (t == (uint32_t)p.G - 1u) {
+                        last = 1;
+                        *p.ticket = 0u;  // leave the counter at zero for the next call
+                    }
+                    *sm.is_last = last;
+                    mbar_arrive(smem_u32(sm.decided));
                 }
+            } else if (lane == 0) {
+                *sm.is_last = 0u;
+                mbar_arrive(smem_u32(sm.decided));
             }
-            *sm.is_last = last;
-            mbar_arrive(smem_u32(sm.decided));
+            last = __shfl_sync(0xffffffffu, last, 0);
+        } else {
+            if (!mbar_wait_bounded(smem_u32(sm.decided), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
+            last = *sm.is_last;
         }
-        if (!mbar_wait_bounded(smem_u32(sm.decided), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
-        if (*sm.is_last == 0u) return;
+        if (last == 0u) return;
         const int nwarps = blockDim.x >> 5;
         uint64_t *tk = reinterpret_cast<uint64_t *>(sm.red + (size_t)p.CWG * p.KW * 32 * VPL) + warp * 64;
         for (int r = warp; r < p.m; r += nwarps) {
