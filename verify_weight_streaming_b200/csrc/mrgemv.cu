@@ -147,6 +147,7 @@ struct Smem {
     uint64_t *cta_done;   // [1] every warp's logits are stored (fused router)
     uint64_t *decided;    // [1] thread 0 knows whether this CTA finished last
     uint32_t *is_last;    // [2]
+    uint64_t *staged;     // [1] the last CTA's copy of the logits is complete
     float *red;           // [CWG][KW][32][VPL]
 };
 
@@ -299,7 +300,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     sm.cta_done = sm.a_full + 1;
     sm.decided = sm.a_full + 2;
     sm.is_last = reinterpret_cast<uint32_t *>(sm.a_full + 3);
-    sm.red = reinterpret_cast<float *>(sm.a_full + 4);
+    sm.staged = sm.a_full + 4;
+    sm.red = reinterpret_cast<float *>(sm.a_full + 6);
 
     // Groups per copy chunk when no slot is refilled (0 when slots are refilled).
     const int chunk_groups = ng <= p.S ? (int)max(1u, (16384u + p.slot_bytes - 1) / p.slot_bytes) : 0;
@@ -329,6 +331,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
         if constexpr (FUSED) {
             mbar_init(smem_u32(sm.cta_done), (uint32_t)(blockDim.x / 32));
             mbar_init(smem_u32(sm.decided), 1);
+            mbar_init(smem_u32(sm.staged), (uint32_t)(blockDim.x / 32));
         }
         if (p.KW > 1) {
             for (int c = 0; c < p.CWG; ++c) {
@@ -451,15 +454,28 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             last = *sm.is_last;
         }
         if (last == 0u) return;
+        // Stage every row's logits in shared memory (the A and ring regions are
+        // free now) with all loads in flight at once, then one warp per row.
         const int nwarps = blockDim.x >> 5;
+        const size_t region = p.a_bytes + (size_t)p.S * p.slot_bytes;
+        const bool staged = (size_t)p.m * p.n * sizeof(float) <= region;
+        float *lg = reinterpret_cast<float *>(smem_raw);
+        if (staged) {
+            const int total = p.m * p.n;
+            for (int e = tid; e < total; e += blockDim.x)
+                lg[e] = __ldcg(p.C + (int64_t)(e / p.n) * p.ldc + (e % p.n));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(sm.staged));
+            if (!mbar_wait_bounded(smem_u32(sm.staged), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
+        }
         uint64_t *tk = reinterpret_cast<uint64_t *>(sm.red + (size_t)p.CWG * p.KW * 32 * VPL) + warp * 64;
         for (int r = warp; r < p.m; r += nwarps) {
-            const float *x = p.C + (int64_t)r * p.ldc;
+            const float *x = staged ? lg + (size_t)r * p.n : p.C + (int64_t)r * p.ldc;
             const uint64_t best = topk::warp_topk_fast<16>(x, p.n, p.topk, lane, 0, 1, 0ull, tk);
             if (lane < p.topk) {
                 const uint32_t j = topk::key_index(best);
                 p.idx[(int64_t)r * p.ldo + lane] = (int32_t)j;
-                if (p.val) p.val[(int64_t)r * p.ldo + lane] = x[j];
+                if (p.val) p.val[(int64_t)r * p.ldo + lane] = topk::selected_value(best, x);
             }
         }
     }
@@ -540,7 +556,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     pl.slot_bytes = (uint32_t)pl.CG * (uint32_t)k * 2u;
     const size_t vpl = (size_t)std::max(1, pl.MB * pl.CG / 32);
     const size_t topk_bytes = fused ? (size_t)kMaxWarps * 64 * 8 : 0;
-    const size_t fixed = topk_bytes + pl.a_bytes + 16 * (size_t)(2 * ng_max + 2 * cwg0) + 32 +
+    const size_t fixed = topk_bytes + pl.a_bytes + 16 * (size_t)(2 * ng_max + 2 * cwg0) + 48 +
                          (size_t)cwg0 * pl.KW * 32 * vpl * 4 + 64;
     const size_t pdl_budget = 110 * 1024;
     const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, (size_t)optin) : (size_t)optin;
@@ -564,7 +580,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
         pl.CWG = std::max(1, std::min(cwg0, s_max / 2));
         pl.S = (s_max / pl.CWG) * pl.CWG;
     }
-    pl.smem = topk_bytes + pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 16 * (size_t)(pl.S + pl.CWG) + 32 +
+    pl.smem = topk_bytes + pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 16 * (size_t)(pl.S + pl.CWG) + 48 +
               (size_t)pl.CWG * pl.KW * 32 * vpl * 4;
     if (pl.smem > (size_t)optin) return MR_ERR_UNSUPPORTED;
     return MR_OK;

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float *__restri
         if (lane < K) {
             const uint32_t j = key_index(best);
             idx[row * ldo + lane] = (int32_t)j;
-            if (val) val[row * ldo + lane] = x[j];
+            if (val) val[row * ldo + lane] = selected_value(best, x);
         }
     }
 }

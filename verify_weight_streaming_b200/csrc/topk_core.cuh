@@ -28,6 +28,24 @@ __device__ __forceinline__ uint64_t make_key(float v, uint32_t idx) {
 
 __device__ __forceinline__ uint32_t key_index(uint64_t key) { return 0xFFFFFFFFu - (uint32_t)key; }
 
+// The logit a key was made from, bit for bit, except where make_key merged
+// values: a zero key stands for +0.0 or -0.0 and the maximal key for any NaN.
+// `exact` is false for those two, and the caller must re-read the value.
+__device__ __forceinline__ float key_value(uint64_t key, bool &exact) {
+    const uint32_t hi = (uint32_t)(key >> 32);
+    exact = hi != 0x80000000u && hi != 0xFFFFFFFFu;
+    const uint32_t b = (hi & 0x80000000u) ? (hi & 0x7FFFFFFFu) : ~hi;
+    return __uint_as_float(b);
+}
+
+// Value to report for a selected key: decoded from the key when that is
+// exact, else re-read from the row.
+__device__ __forceinline__ float selected_value(uint64_t key, const float *x) {
+    bool exact;
+    const float v = key_value(key, exact);
+    return exact ? v : x[key_index(key)];
+}
+
 // Sort L keys descending (insertion network, compile-time indices).
 template <int L>
 __device__ __forceinline__ void sort_desc(uint64_t (&x)[L]) {
@@ -105,9 +123,15 @@ __device__ __forceinline__ int warp_rank(uint64_t key, int lane) {
 template <int P>
 __device__ __forceinline__ uint64_t warp_topk_merge(uint64_t (&key)[P], uint64_t run, int K, int lane,
                                                     uint64_t *scratch) {
-    uint64_t mx = run;
+    // Lane maximum by a pairwise tree (short dependency chain).
+    uint64_t t[P];
 #pragma unroll
-    for (int i = 0; i < P; ++i) mx = key[i] > mx ? key[i] : mx;
+    for (int i = 0; i < P; ++i) t[i] = key[i];
+#pragma unroll
+    for (int w = 1; w < P; w <<= 1)
+#pragma unroll
+        for (int i = 0; i + w < P; i += 2 * w) t[i] = t[i + w] > t[i] ? t[i + w] : t[i];
+    const uint64_t mx = t[0] > run ? t[0] : run;
     const int r0 = warp_rank(mx, lane);
     const unsigned who = __ballot_sync(0xffffffffu, r0 == K - 1 && mx != 0ull);
     // Fewer than K nonzero lane maxima: every nonzero key is a candidate.
