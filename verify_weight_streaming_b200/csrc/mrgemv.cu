@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
         if constexpr (FUSED) {
             mbar_init(smem_u32(sm.cta_done), (uint32_t)(blockDim.x / 32));
             mbar_init(smem_u32(sm.decided), 1);
-            mbar_init(smem_u32(sm.staged), (uint32_t)(blockDim.x / 32));
+            mbar_init(smem_u32(sm.staged), 1);
         }
         if (p.KW > 1) {
             for (int c = 0; c < p.CWG; ++c) {
@@ -455,17 +455,27 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
         }
         if (last == 0u) return;
         // Stage every row's logits in shared memory (the A and ring regions are
-        // free now) with all loads in flight at once, then one warp per row.
+        // free now) with one bulk copy per row, all in flight together, when
+        // the rows are 16-byte aligned; otherwise read them from global memory.
         const int nwarps = blockDim.x >> 5;
         const size_t region = p.a_bytes + (size_t)p.S * p.slot_bytes;
-        const bool staged = (size_t)p.m * p.n * sizeof(float) <= region;
+        const uint32_t row_bytes = (uint32_t)p.n * 4u;
+        const bool staged = (size_t)p.m * row_bytes <= region && (row_bytes & 15u) == 0 &&
+                            ((uintptr_t)p.C & 15u) == 0 && (p.ldc & 3) == 0;
         float *lg = reinterpret_cast<float *>(smem_raw);
         if (staged) {
-            const int total = p.m * p.n;
-            for (int e = tid; e < total; e += blockDim.x)
-                lg[e] = __ldcg(p.C + (int64_t)(e / p.n) * p.ldc + (e % p.n));
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(sm.staged));
+            if (warp == 0) {
+                if (lane == 0) {
+                    // The logits were written by other CTAs through the generic
+                    // proxy; order them before the async-proxy reads.
+                    asm volatile("fence.proxy.async;" ::: "memory");
+                    const uint32_t bar = smem_u32(sm.staged);
+                    mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)p.m);
+                    for (int r = 0; r < p.m; ++r)
+                        bulk_g2s(smem_u32(lg + (size_t)r * p.n), p.C + (int64_t)r * p.ldc, row_bytes, bar);
+                }
+                __syncwarp();
+            }
             if (!mbar_wait_bounded(smem_u32(sm.staged), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
         }
         uint64_t *tk = reinterpret_cast<uint64_t *>(sm.red + (size_t)p.CWG * p.KW * 32 * VPL) + warp * 64;
