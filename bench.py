@@ -63,13 +63,19 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+# Source files whose change invalidates a recorded ncu traffic figure.
+KERNEL_SOURCES = {
+    "gemv_router": ("mrgemv.cu", "common.cuh", "topk_core.cuh"),
+    "gemm": ("gemm_f16.cu", "common.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str = "gemv_router") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "verify_weight_streaming_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -80,7 +86,7 @@ def recorded_traffic(kernel: str):
         with open(path) as f:
             rec = json.load(f)
         entry = rec[kernel]
-        if entry.get("source_hash") != kernel_source_hash():
+        if entry.get("source_hash") != kernel_source_hash(kernel):
             return None
         return float(entry["dram_bytes_per_launch"])
     except Exception:
