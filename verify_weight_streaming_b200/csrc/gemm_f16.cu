@@ -5,9 +5,11 @@
 // tiles (M % 128 in 1..64), and outputs that are bitwise identical whatever
 // tile is chosen.  Rebuilt for B200:
 //
-//  * one CTA per 128 x BN output tile, 6 warps: warp 0 issues TMA loads, warp
-//    1 owns the tensor memory and issues tcgen05.mma from one thread, warps
-//    2..5 drain the accumulator (tcgen05.ld) and store the tile;
+//  * persistent CTAs (one per SM) walk the 128 x BN output tiles; 6 warps:
+//    warp 0 issues TMA loads, warp 1 owns the tensor memory and issues
+//    tcgen05.mma from one thread, warps 2..5 drain the accumulator
+//    (tcgen05.ld) and store the tile.  Two accumulator buffers in tensor
+//    memory let one tile's epilogue run under the next tile's MMAs;
 //  * A and Wt tiles of 64 K-elements (one 128-byte swizzle atom per row) are
 //    loaded by TMA (no multicast) into a ring of STAGES shared-memory stages,
 //    full/empty mbarriers between the producer and the MMA thread;
@@ -41,7 +43,7 @@ constexpr uint32_t kABytes = BM * BK * 2;
 struct TileDesc {
     int bn;
     int stages;
-    int tmem_cols;
+    int acc_cols;   // tensor-memory columns per accumulator buffer (power of two >= bn)
     const char *name;
 };
 
@@ -169,11 +171,15 @@ __device__ __forceinline__ void store16(void *C, int64_t ldc, int row, int col, 
 
 // ---- the kernel --------------------------------------------------------------
 
-template <int BN, int STAGES, int TMEM_COLS, int OUT>
+template <int BN, int STAGES, int ACC_COLS, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, void *C,
                 int64_t ldc, int M, int N, int K, uint32_t idesc) {
+    // Persistent: CTA b takes tiles b, b + gridDim.x, ... (N-tiles fastest).
+    // Two accumulator buffers of ACC_COLS tensor-memory columns each: the
+    // epilogue drains tile i from one while the MMAs of tile i+1 fill the other.
     constexpr uint32_t kBBytes = (uint32_t)BN * BK * 2;
+    constexpr uint32_t kTmemCols = 2 * ACC_COLS;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -181,15 +187,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sA = base;
     const uint32_t sB = base + STAGES * kABytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + STAGES * (kABytes + kBBytes));
-    uint64_t *full = bars;
-    uint64_t *empty = bars + STAGES;
-    uint64_t *tmem_full = bars + 2 * STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 1);
+    uint64_t *full = bars;                    // [STAGES] TMA -> MMA
+    uint64_t *empty = bars + STAGES;          // [STAGES] MMA -> TMA
+    uint64_t *acc_full = bars + 2 * STAGES;   // [2] MMA -> epilogue
+    uint64_t *acc_empty = bars + 2 * STAGES + 2;  // [2] epilogue -> MMA
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * BM;
-    const int n0 = blockIdx.x * BN;
+    const int ntn = (N + BN - 1) / BN;
+    const int ntiles = ((M + BM - 1) / BM) * ntn;
     const int nkb = (K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
@@ -197,12 +204,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&full[s]), 1);
             mbar_init(smem_u32(&empty[s]), 1);
         }
-        mbar_init(smem_u32(tmem_full), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&acc_full[b]), 1);
+            mbar_init(smem_u32(&acc_empty[b]), 4);  // one arrival per epilogue warp
+        }
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
     }
-    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -212,54 +222,78 @@ __global__ void __launch_bounds__(kThreads, 1)
     // same barrier) and let lane 0 issue: a lone lane spinning in try_wait
     // beside warp-mates parked elsewhere can stall for the suspend limit.
     if (warp == 0) {
-        // Producer: stage s is reused after the MMAs reading it complete.
-        for (int kb = 0; kb < nkb; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t par = ((uint32_t)(kb / STAGES) & 1u) ^ 1u;
-            if (!mbar_wait_bounded(smem_u32(&empty[s]), par, MR_DEVERR_GEMM_TIMEOUT)) break;
-            if (lane == 0) {
-                const uint32_t fb = smem_u32(&full[s]);
-                mbar_arrive_expect_tx(fb, kABytes + kBBytes);
-                tma_load_2d(sA + s * kABytes, &tmA, kb * BK, m0, fb);
-                tma_load_2d(sB + s * kBBytes, &tmB, kb * BK, n0, fb);
+        // Producer: k-block `it` counts across tiles, so stages and phases
+        // continue from one tile to the next.
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const int m0 = (t / ntn) * BM, n0 = (t % ntn) * BN;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const uint32_t s = it % STAGES;
+                const uint32_t par = ((it / STAGES) & 1u) ^ 1u;
+                ok = mbar_wait_bounded(smem_u32(&empty[s]), par, MR_DEVERR_GEMM_TIMEOUT);
+                if (!ok) break;
+                if (lane == 0) {
+                    const uint32_t fb = smem_u32(&full[s]);
+                    mbar_arrive_expect_tx(fb, kABytes + kBBytes);
+                    tma_load_2d(sA + s * kABytes, &tmA, kb * BK, m0, fb);
+                    tma_load_2d(sB + s * kBBytes, &tmB, kb * BK, n0, fb);
+                }
+                __syncwarp();
             }
-            __syncwarp();
         }
     } else if (warp == 1) {
+        uint32_t it = 0, ti = 0;
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t par = (uint32_t)(kb / STAGES) & 1u;
-            ok = mbar_wait_bounded(smem_u32(&full[s]), par, MR_DEVERR_GEMM_TIMEOUT);
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++ti) {
+            const uint32_t b = ti & 1u;
+            // Wait until the epilogue has drained this buffer's previous tile.
+            ok = mbar_wait_bounded(smem_u32(&acc_empty[b]), ((ti >> 1) & 1u) ^ 1u, MR_DEVERR_GEMM_TIMEOUT);
             if (!ok) break;
             tc_fence_after();
-            if (lane == 0) {
+            const uint32_t acc = tmem + b * ACC_COLS;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const uint32_t s = it % STAGES;
+                const uint32_t par = (it / STAGES) & 1u;
+                ok = mbar_wait_bounded(smem_u32(&full[s]), par, MR_DEVERR_GEMM_TIMEOUT);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk) {
-                    const uint64_t ad = sw128_desc(sA + s * kABytes + kk * 32);
-                    const uint64_t bd = sw128_desc(sB + s * kBBytes + kk * 32);
-                    mma_f16(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t ad = sw128_desc(sA + s * kABytes + kk * 32);
+                        const uint64_t bd = sw128_desc(sB + s * kBBytes + kk * 32);
+                        mma_f16(acc, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(smem_u32(&empty[s]));
                 }
-                mma_commit(smem_u32(&empty[s]));
+                __syncwarp();
             }
+            if (ok && lane == 0) mma_commit(smem_u32(&acc_full[b]));
             __syncwarp();
         }
-        if (ok && lane == 0) mma_commit(smem_u32(tmem_full));
-        __syncwarp();
     } else {
         // Epilogue warps 2..5: warp w reads tensor-memory lanes 32*(w%4) .. +31.
         const int q = warp & 3;
-        const int row = m0 + 32 * q + lane;
-        const bool ok = mbar_wait_bounded(smem_u32(tmem_full), 0u, MR_DEVERR_GEMM_TIMEOUT);
-        tc_fence_after();
-        if (ok) {
+        uint32_t ti = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++ti) {
+            const uint32_t b = ti & 1u;
+            const int m0 = (t / ntn) * BM, n0 = (t % ntn) * BN;
+            const int row = m0 + 32 * q + lane;
+            if (!mbar_wait_bounded(smem_u32(&acc_full[b]), (ti >> 1) & 1u, MR_DEVERR_GEMM_TIMEOUT)) break;
+            tc_fence_after();
+            const uint32_t acc = tmem + b * ACC_COLS + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
             for (int c = 0; c < BN / 16; ++c) {
                 uint32_t r[16];
-                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * 16), r);
+                tmem_ld16(acc + (uint32_t)(c * 16), r);
                 const int col = n0 + c * 16;
                 if (row < M && col < N) store16<OUT>(C, ldc, row, col, N, r);
             }
+            // This warp's lanes of the buffer are read: let the MMAs reuse it.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
         }
     }
 
@@ -267,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -277,7 +311,7 @@ using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, void *, int64_t,
 
 template <int T, int OUT>
 constexpr KernelFn kernel_of() {
-    return gemm_kernel<kTiles[T].bn, kTiles[T].stages, kTiles[T].tmem_cols, OUT>;
+    return gemm_kernel<kTiles[T].bn, kTiles[T].stages, kTiles[T].acc_cols, OUT>;
 }
 
 template <int OUT>
@@ -346,26 +380,32 @@ uint32_t make_idesc(int in_dtype, int bn) {
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
-// Tile selection: estimated time = waves x per-tile time, where a wave is one
-// CTA per SM, per-tile time is the padded MMA work of the tile at a rate that
-// grows with BN (wider tiles reuse each A stage for more columns) plus a fixed
-// prologue / epilogue cost.  Row tails are counted as whole 128-row tiles, so
-// an M whose M % 128 is small pays for the padding it creates; narrow N (the
-// N = 96 projections) favours tiles that divide N and spread over more SMs.
+// Tile selection: estimated time = waves x per-tile time, a wave being one
+// tile on every active SM.  Per-tile time is the larger of
+//  * the padded MMA work of the tile at a rate that grows with BN (wider tiles
+//    reuse each A stage for more columns) plus a small fixed cost, and
+//  * streaming the tile's operands into the SM, (128 + BN) x K x 2 bytes, at
+//    the per-SM share of the measured copy bandwidth (at most ~100 GB/s per SM).
+// Row tails count as whole 128-row tiles, so an M with a small M % 128 pays for
+// the padding it creates (the audit's tail-tile rule); narrow N (the N = 96
+// projections) is bounded by the operand stream and favours spreading tiles
+// over more SMs.
 int select_tile(int M, int N, int K, int sms) {
     if (M < 1 || N < 1 || K < 1 || sms < 1) return -1;
     const double eff[kNumTiles] = {0.30, 0.55, 0.70, 0.80, 0.88, 0.92};
     const double per_sm_flops_us = 1.6e15 / 148.0 * 1e-6;   // dense f16 per SM per microsecond
+    const double hbm_bytes_us = 6.5e6;                       // ~6.5 TB/s in bytes per microsecond
     int best = -1;
     double best_t = 1e300;
     for (int t = 0; t < kNumTiles; ++t) {
         const int bn = kTiles[t].bn;
         const int64_t tiles = (int64_t)((M + BM - 1) / BM) * ((N + bn - 1) / bn);
+        const int64_t active = std::min<int64_t>(tiles, sms);
         const int64_t waves = (tiles + sms - 1) / sms;
         const double kpad = (double)((K + BK - 1) / BK * BK);
-        const double tile_us = 2.0 * BM * bn * kpad / (per_sm_flops_us * eff[t]) + 1.5;
-        // A tile streamed per CTA bounds narrow tiles: bytes per CTA at ~150 GB/s.
-        const double stream_us = (BM + bn) * kpad * 2.0 / 150e3;
+        const double tile_us = 2.0 * BM * bn * kpad / (per_sm_flops_us * eff[t]) + 0.3;
+        const double sm_bw = std::min(1.0e5, hbm_bytes_us / (double)active);
+        const double stream_us = (BM + bn) * kpad * 2.0 / sm_bw;
         const double t_est = (double)waves * std::max(tile_us, stream_us);
         if (t_est < best_t * 0.999) {
             best_t = t_est;
@@ -419,7 +459,8 @@ extern "C" mr_status gemm_f16(const void *A, int64_t lda, const void *Wt, int64_
     if (!encode_operand(&tb, Wt, N, K, ldw, in_dtype, td.bn)) return MR_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((N + td.bn - 1) / td.bn), (unsigned)((M + BM - 1) / BM));
+    const int64_t ntiles = (int64_t)((N + td.bn - 1) / td.bn) * ((M + BM - 1) / BM);
+    cfg.gridDim = dim3((unsigned)std::min<int64_t>(ntiles, sms > 0 ? sms : 148));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem_bytes_for(td.bn, td.stages);
     cfg.stream = static_cast<cudaStream_t>(stream);
