@@ -646,9 +646,15 @@ def gemm_sweep(quick=False):
         C = torch.empty((M, 96), dtype=torch.float16, device="cuda")
         calls = [(lambda W=w96[i]: mr.gemm_f16(a16, W, C)) for i in range(36)]
         us = _time_calls(torch, calls)
+        Cs = [torch.empty((M, 96), dtype=torch.float16, device="cuda") for _ in range(36)]
+        ug = _time_calls(torch, [lambda: mr.gemm_f16_grouped(a16, w96, Cs)] * 4)
         out["narrow"][str(M)] = {"us_per_call": us, "us_per_36_calls": 36 * us,
                                  "TFLOPs": 2.0 * M * 96 * K / (us * 1e-6) / 1e12,
-                                 "tile": mr.gemm_f16_tile_name(mr.gemm_f16_select_tile(M, 96, K))}
+                                 "tile": mr.gemm_f16_tile_name(mr.gemm_f16_select_tile(M, 96, K)),
+                                 "grouped_us_for_36": ug,
+                                 "grouped_TFLOPs": 36 * 2.0 * M * 96 * K / (ug * 1e-6) / 1e12,
+                                 "grouped_tile": mr.gemm_f16_tile_name(
+                                     mr.gemm_f16_grouped_select_tile(M, 96, K, 36))}
     out["summary"] = {"tflops_M_ge_1024_mean": float(np.mean(big)) if big else None,
                       "tflops_M_ge_1024_max": float(np.max(big)) if big else None,
                       "peak_bf16_tflops": tf_burst, "peak_kind": kind,

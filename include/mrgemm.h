@@ -207,6 +207,29 @@ mr_status gemm_f16(const void *A, int64_t lda, const void *Wt, int64_t ldw,
                    int32_t in_dtype, int32_t out_dtype, int32_t tile_id,
                    void *stream);
 
+/*
+ * gemm_f16_grouped -- G GEMMs that share A in one launch: for g < G,
+ *   Cs[g][i][j] = sum_p A[i][p] * Wts[g][j][p]
+ * The 36 independent N = 96 projections of one prompt chunk in the
+ * "opus r35 track A" audit (section 2, Walbe table: N = 96, K = 2560, 36
+ * calls) are this shape.  Each output has exactly the bits gemm_f16 gives for
+ * (A, Wts[g]) with any tile: every tile runs the same K sequence.  When N is a
+ * multiple of 16 that divides the tile width, one tile covers several groups
+ * (for N = 96, two groups per 192-column tile), so A is streamed once for
+ * them.
+ *
+ * Wts, Cs : HOST arrays of G device pointers (Wts[g]: N rows of K elements,
+ *           stride ldw; Cs[g]: M rows of N elements, stride ldc).
+ * 1 <= G <= 64 (MR_ERR_UNSUPPORTED above); other arguments as gemm_f16.
+ */
+mr_status gemm_f16_grouped(const void *A, int64_t lda, const void *const *Wts, int64_t ldw,
+                           void *const *Cs, int64_t ldc, int32_t M, int32_t N, int32_t K,
+                           int32_t G, int32_t in_dtype, int32_t out_dtype, int32_t tile_id,
+                           void *stream);
+
+/* The tile gemm_f16_grouped picks for (M, N, K, G) when tile_id is -1. */
+int32_t gemm_f16_grouped_select_tile(int32_t M, int32_t N, int32_t K, int32_t G);
+
 /* Number of tile shapes gemm_f16 can run. */
 int32_t gemm_f16_num_tiles(void);
 

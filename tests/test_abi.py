@@ -131,3 +131,19 @@ def test_fused_router_workspace_bytes():
     assert mr.router_gemv_topk_workspace_bytes(4, 512, False) == 256 + 4 * 512 * 4
     assert mr.router_gemv_topk_workspace_bytes(0, 512, False) == 0
     assert fused(logits=P(1024), wsb=256) == mr.MR_ERR_CUDA  # valid; no device here
+
+
+def test_grouped_validation():
+    W = (P * 2)(256, 256)
+    C = (P * 2)(256, 256)
+    g = mr.lib.gemm_f16_grouped
+    assert g(A16, 64, W, 64, C, 32, 4, 32, 64, 0, 0, 0, -1, None) == mr.MR_ERR_INVALID_ARG
+    W65 = (P * 65)(*([256] * 65))
+    C65 = (P * 65)(*([256] * 65))
+    assert g(A16, 64, W65, 64, C65, 32, 4, 32, 64, 65, 0, 0, -1, None) == mr.MR_ERR_UNSUPPORTED
+    Wn = (P * 2)(256, None)
+    assert g(A16, 64, Wn, 64, C, 32, 4, 32, 64, 2, 0, 0, -1, None) == mr.MR_ERR_INVALID_ARG
+    Wb = (P * 2)(256, 258)
+    assert g(A16, 64, Wb, 64, C, 32, 4, 32, 64, 2, 0, 0, -1, None) == mr.MR_ERR_MISALIGNED
+    assert g(A16, 64, W, 64, C, 32, 4, 32, 64, 2, 0, 0, -1, None) == mr.MR_ERR_CUDA  # valid; no device
+    assert 0 <= mr.gemm_f16_grouped_select_tile(2048, 96, 2560, 36) < mr.gemm_f16_num_tiles()

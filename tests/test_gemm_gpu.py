@@ -156,3 +156,43 @@ def test_selector_choices_are_valid():
         for N in (96, 512, 640, 1152, 1664, 4096, 6144):
             t = mr.gemm_f16_select_tile(M, N, 2560)
             assert 0 <= t < mr.gemm_f16_num_tiles()
+
+
+def run_grouped(a_bits, w_list, fmt="f16", out_fmt="f16", tile=-1):
+    M, K = a_bits.shape
+    N = w_list[0].shape[0]
+    A = dev_bits(a_bits, TORCH_DT[fmt])
+    Ws = [dev_bits(w, TORCH_DT[fmt]) for w in w_list]
+    ldc = (N + 7) // 8 * 8
+    bufs = [torch.full((M + 1, ldc), float("nan"), dtype=TORCH_DT[out_fmt], device="cuda") for _ in w_list]
+    mr.gemm_f16_grouped(A, Ws, [b[:M, :N] for b in bufs], tile_id=tile)
+    out = []
+    for b in bufs:
+        f = host(b.float())
+        assert np.isnan(f[M]).all() and np.isnan(f[:M, N:]).all(), "write outside C"
+        out.append(host(b.view(torch.int16) if out_fmt != "f32" else b.view(torch.int32))[:M, :N])
+    return out
+
+
+@pytest.mark.parametrize("M", [512, 1983])
+def test_grouped_36_narrow_matches_single_calls(M):
+    """The audit's chunk: one A, 36 W[96, 2560]; every output equals its single call."""
+    a = synth.narrow(M)[0]
+    ws = [synth.narrow(1, w_index=i)[1] for i in range(36)]
+    grouped = run_grouped(a, ws)
+    for i in (0, 1, 17, 35):
+        _, ref = run_gemm(a, ws[i])
+        assert np.array_equal(grouped[i], ref), f"group {i}"
+    c = synth.bits_to_float32(grouped[7].view(np.uint16), "f16")
+    check(c, a, ws[7], "f16", "f16")
+
+
+@pytest.mark.parametrize("G,N,K", [(5, 48, 200), (3, 40, 136), (2, 300, 72), (1, 96, 2560), (64, 16, 64)])
+def test_grouped_every_tile_bitwise(G, N, K):
+    a = synth.normal_bits(61 + G, (257, K), "bf16", 1.0)
+    ws = [synth.normal_bits(62 + 7 * g + N, (N, K), "bf16", 1.0 / np.sqrt(K)) for g in range(G)]
+    refs = [run_gemm(a, w, in_fmt="bf16", out_fmt="bf16", tile=0)[1] for w in ws]
+    for tile in range(-1, mr.gemm_f16_num_tiles()):
+        outs = run_grouped(a, ws, fmt="bf16", out_fmt="bf16", tile=tile)
+        for g in range(G):
+            assert np.array_equal(outs[g], refs[g]), (tile, g)

@@ -21,7 +21,8 @@ MR_DEVERR_GEMV_TIMEOUT, MR_DEVERR_GEMM_TIMEOUT, MR_DEVERR_TOPK_TIMEOUT, MR_DEVER
 
 EXPORTS = (
     "mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
-    "router_gemv_topk_workspace_bytes", "router_gemv_topk_noalloc", "router_gemv_topk_noalloc_max_logits", "gemm_f16", "gemm_f16_num_tiles",
+    "router_gemv_topk_workspace_bytes", "router_gemv_topk_noalloc", "router_gemv_topk_noalloc_max_logits", "gemm_f16_grouped",
+    "gemm_f16_grouped_select_tile", "gemm_f16", "gemm_f16_num_tiles",
     "gemm_f16_tile_name", "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout",
     "mr_status_str", "mr_version",
 )
@@ -56,6 +57,8 @@ def _load() -> ctypes.CDLL:
     L.router_gemv_topk_noalloc_max_logits.argtypes = []
     L.router_gemv_topk_noalloc_max_logits.restype = ctypes.c_size_t
     L.gemm_f16.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, I32, I32, P]
+    L.gemm_f16_grouped.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, I32, I32, I32, P]
+    L.gemm_f16_grouped_select_tile.argtypes = [I32, I32, I32, I32]
     L.gemm_f16_num_tiles.argtypes = []
     L.gemm_f16_tile_name.argtypes = [I32]
     L.gemm_f16_tile_name.restype = ctypes.c_char_p
@@ -67,7 +70,7 @@ def _load() -> ctypes.CDLL:
     L.mr_version.argtypes = []
     L.mr_version.restype = ctypes.c_char_p
     for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
-                 "router_gemv_topk_noalloc", "gemm_f16", "gemm_f16_num_tiles",
+                 "router_gemv_topk_noalloc", "gemm_f16_grouped", "gemm_f16_grouped_select_tile", "gemm_f16", "gemm_f16_num_tiles",
                  "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     return L
@@ -200,6 +203,29 @@ def gemm_f16(A, Wt, C, tile_id: int = -1, in_dtype: int | None = None, stream=No
     st = lib.gemm_f16(A.data_ptr(), lda, Wt.data_ptr(), ldw, C.data_ptr(), ldc, M, N, K,
                       idt, _dtype_code(C), tile_id, _stream(stream))
     _check(st, "gemm_f16")
+
+
+def gemm_f16_grouped(A, Wts, Cs, tile_id: int = -1, in_dtype: int | None = None, stream=None) -> None:
+    """Cs[g] = A . Wts[g]^T for every g in one launch (lists of equal-shape tensors)."""
+    M, K, lda = _rows(A, "A")
+    if len(Wts) != len(Cs) or not Wts:
+        raise ValueError("Wts and Cs must be non-empty lists of the same length")
+    N, kw, ldw = _rows(Wts[0], "Wts[0]")
+    _, _, ldc = _rows(Cs[0], "Cs[0]")
+    for w, c in zip(Wts, Cs):
+        if tuple(w.shape) != (N, K) or w.stride(0) != ldw or tuple(c.shape) != (M, N) or c.stride(0) != ldc:
+            raise ValueError("every Wts[g] must be [N,K] and every Cs[g] [M,N] with common strides")
+    G = len(Wts)
+    wp = (ctypes.c_void_p * G)(*[w.data_ptr() for w in Wts])
+    cp = (ctypes.c_void_p * G)(*[c.data_ptr() for c in Cs])
+    idt = _dtype_code(A) if in_dtype is None else in_dtype
+    st = lib.gemm_f16_grouped(A.data_ptr(), lda, wp, ldw, cp, ldc, M, N, K, G, idt, _dtype_code(Cs[0]),
+                              tile_id, _stream(stream))
+    _check(st, "gemm_f16_grouped")
+
+
+def gemm_f16_grouped_select_tile(M: int, N: int, K: int, G: int) -> int:
+    return int(lib.gemm_f16_grouped_select_tile(M, N, K, G))
 
 
 def gemm_f16_num_tiles() -> int:

@@ -30,6 +30,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 namespace mr {
@@ -171,11 +172,28 @@ __device__ __forceinline__ void store16(void *C, int64_t ldc, int row, int col, 
 
 // ---- the kernel --------------------------------------------------------------
 
-template <int BN, int STAGES, int ACC_COLS, int OUT>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, void *C,
-                int64_t ldc, int M, int N, int K, uint32_t idesc) {
-    // Persistent: CTA b takes tiles b, b + gridDim.x, ... (N-tiles fastest).
+// Up to MAXG weight matrices ("groups") that share A, each with its own
+// tensor map and output.  A tile covers either BN columns of one group
+// (P == 1, tn_per_group tiles per group) or P whole groups of N columns each
+// (P > 1, BN == P * N, N a multiple of 16).
+template <int MAXG>
+struct GemmArgs {
+    CUtensorMap tmA;
+    CUtensorMap tmB[MAXG];
+    void *C[MAXG];
+    int64_t ldc;
+    int M, N, K;
+    int G, P, tn_per_group, ntn;
+    uint32_t idesc;
+};
+
+template <int BN, int STAGES, int ACC_COLS, int OUT, int MAXG>
+__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs<MAXG> args) {
+    const CUtensorMap &tmA = args.tmA;
+    const int M = args.M, N = args.N, K = args.K, G = args.G, P = args.P;
+    const int64_t ldc = args.ldc;
+    const uint32_t idesc = args.idesc;
+    // Persistent: CTA b takes tiles b, b + gridDim.x, ... (N-tile slots fastest).
     // Two accumulator buffers of ACC_COLS tensor-memory columns each: the
     // epilogue drains tile i from one while the MMAs of tile i+1 fill the other.
     constexpr uint32_t kBBytes = (uint32_t)BN * BK * 2;
@@ -195,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int ntn = (N + BN - 1) / BN;
+    const int ntn = args.ntn;
     const int ntiles = ((M + BM - 1) / BM) * ntn;
     const int nkb = (K + BK - 1) / BK;
 
@@ -210,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_mbar_init();
         prefetch_tmap(&tmA);
-        prefetch_tmap(&tmB);
+        if (MAXG == 1) prefetch_tmap(&args.tmB[0]);
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tc_fence_before();
@@ -227,7 +245,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const int m0 = (t / ntn) * BM, n0 = (t % ntn) * BN;
+            const int m0 = (t / ntn) * BM, slot = t % ntn;
+            // Groups of this tile and the B rows each contributes.
+            const int g0 = P > 1 ? slot * P : slot / args.tn_per_group;
+            const int ng = P > 1 ? min(P, G - g0) : 1;
+            const int n0 = P > 1 ? 0 : (slot % args.tn_per_group) * BN;
+            const uint32_t b_rows = P > 1 ? (uint32_t)N : (uint32_t)BN;
+            const uint32_t tx = kABytes + (uint32_t)ng * b_rows * BK * 2;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const uint32_t s = it % STAGES;
                 const uint32_t par = ((it / STAGES) & 1u) ^ 1u;
@@ -235,9 +259,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 if (lane == 0) {
                     const uint32_t fb = smem_u32(&full[s]);
-                    mbar_arrive_expect_tx(fb, kABytes + kBBytes);
+                    mbar_arrive_expect_tx(fb, tx);
                     tma_load_2d(sA + s * kABytes, &tmA, kb * BK, m0, fb);
-                    tma_load_2d(sB + s * kBBytes, &tmB, kb * BK, n0, fb);
+                    for (int j = 0; j < ng; ++j)
+                        tma_load_2d(sB + s * kBBytes + (uint32_t)j * b_rows * BK * 2, &args.tmB[g0 + j], kb * BK,
+                                    n0, fb);
                 }
                 __syncwarp();
             }
@@ -278,7 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ti = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++ti) {
             const uint32_t b = ti & 1u;
-            const int m0 = (t / ntn) * BM, n0 = (t % ntn) * BN;
+            const int m0 = (t / ntn) * BM, slot = t % ntn;
+            const int g0 = P > 1 ? slot * P : slot / args.tn_per_group;
+            const int n0 = P > 1 ? 0 : (slot % args.tn_per_group) * BN;
             const int row = m0 + 32 * q + lane;
             if (!mbar_wait_bounded(smem_u32(&acc_full[b]), (ti >> 1) & 1u, MR_DEVERR_GEMM_TIMEOUT)) break;
             tc_fence_after();
@@ -287,8 +315,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < BN / 16; ++c) {
                 uint32_t r[16];
                 tmem_ld16(acc + (uint32_t)(c * 16), r);
-                const int col = n0 + c * 16;
-                if (row < M && col < N) store16<OUT>(C, ldc, row, col, N, r);
+                // Column c*16 of the tile: group and column within the group.
+                const int g = P > 1 ? g0 + (c * 16) / N : g0;
+                const int col = P > 1 ? (c * 16) % N : n0 + c * 16;
+                if (row < M && col < N && g < G) store16<OUT>(args.C[g], ldc, row, col, N, r);
             }
             // This warp's lanes of the buffer are read: let the MMAs reuse it.
             tc_fence_before();
@@ -307,29 +337,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- host side -------------------------------------------------------------
 
-using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, void *, int64_t, int, int, int, uint32_t);
+constexpr int kMaxGroups = 64;
 
-template <int T, int OUT>
-constexpr KernelFn kernel_of() {
-    return gemm_kernel<kTiles[T].bn, kTiles[T].stages, kTiles[T].acc_cols, OUT>;
+template <int MAXG>
+using KernelFn = void (*)(const GemmArgs<MAXG>);
+
+template <int T, int OUT, int MAXG>
+constexpr KernelFn<MAXG> kernel_of() {
+    return gemm_kernel<kTiles[T].bn, kTiles[T].stages, kTiles[T].acc_cols, OUT, MAXG>;
 }
 
-template <int OUT>
-KernelFn pick_out(int t) {
+template <int OUT, int MAXG>
+KernelFn<MAXG> pick_out(int t) {
     switch (t) {
-        case 0: return kernel_of<0, OUT>();
-        case 1: return kernel_of<1, OUT>();
-        case 2: return kernel_of<2, OUT>();
-        case 3: return kernel_of<3, OUT>();
-        case 4: return kernel_of<4, OUT>();
-        default: return kernel_of<5, OUT>();
+        case 0: return kernel_of<0, OUT, MAXG>();
+        case 1: return kernel_of<1, OUT, MAXG>();
+        case 2: return kernel_of<2, OUT, MAXG>();
+        case 3: return kernel_of<3, OUT, MAXG>();
+        case 4: return kernel_of<4, OUT, MAXG>();
+        default: return kernel_of<5, OUT, MAXG>();
     }
 }
 
-KernelFn kernel_for(int tile, int out) {
-    if (out == MR_F16) return pick_out<MR_F16>(tile);
-    if (out == MR_BF16) return pick_out<MR_BF16>(tile);
-    return pick_out<MR_F32>(tile);
+template <int MAXG>
+KernelFn<MAXG> kernel_for(int tile, int out) {
+    if (out == MR_F16) return pick_out<MR_F16, MAXG>(tile);
+    if (out == MR_BF16) return pick_out<MR_BF16, MAXG>(tile);
+    return pick_out<MR_F32, MAXG>(tile);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -349,8 +383,12 @@ cudaError_t init_device(int device) {
     if (device >= 0 && device < 64 && !g_attr_done[device]) {
         for (int t = 0; t < kNumTiles; ++t)
             for (int out = 0; out < 3; ++out) {
-                cudaError_t e = cudaFuncSetAttribute(kernel_for(t, out), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     (int)smem_bytes_for(kTiles[t].bn, kTiles[t].stages));
+                const int smem = (int)smem_bytes_for(kTiles[t].bn, kTiles[t].stages);
+                cudaError_t e = cudaFuncSetAttribute(kernel_for<1>(t, out),
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                if (e != cudaSuccess) return e;
+                e = cudaFuncSetAttribute(kernel_for<kMaxGroups>(t, out), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
                 if (e != cudaSuccess) return e;
             }
         g_attr_done[device] = true;
@@ -390,8 +428,20 @@ uint32_t make_idesc(int in_dtype, int bn) {
 // the padding it creates (the audit's tail-tile rule); narrow N (the N = 96
 // projections) is bounded by the operand stream and favours spreading tiles
 // over more SMs.
-int select_tile(int M, int N, int K, int sms) {
-    if (M < 1 || N < 1 || K < 1 || sms < 1) return -1;
+// Groups packed per tile of width bn: a tile holds whole groups when N
+// divides bn and is a multiple of 16 (so no 16-column chunk straddles two
+// groups); otherwise 1 (a group spans ceil(N / bn) tiles).
+int pack_factor(int bn, int N, int G) {
+    if (G > 1 && N < bn && bn % N == 0 && N % 16 == 0) return bn / N;
+    return 1;
+}
+
+int64_t n_slots(int bn, int N, int G, int P) {
+    return P > 1 ? (int64_t)((G + P - 1) / P) : (int64_t)G * ((N + bn - 1) / bn);
+}
+
+int select_tile_grouped(int M, int N, int K, int G, int sms) {
+    if (M < 1 || N < 1 || K < 1 || G < 1 || sms < 1) return -1;
     const double eff[kNumTiles] = {0.30, 0.55, 0.70, 0.80, 0.88, 0.92};
     const double per_sm_flops_us = 1.6e15 / 148.0 * 1e-6;   // dense f16 per SM per microsecond
     const double hbm_bytes_us = 6.5e6;                       // ~6.5 TB/s in bytes per microsecond
@@ -399,7 +449,8 @@ int select_tile(int M, int N, int K, int sms) {
     double best_t = 1e300;
     for (int t = 0; t < kNumTiles; ++t) {
         const int bn = kTiles[t].bn;
-        const int64_t tiles = (int64_t)((M + BM - 1) / BM) * ((N + bn - 1) / bn);
+        const int P = pack_factor(bn, N, G);
+        const int64_t tiles = (int64_t)((M + BM - 1) / BM) * n_slots(bn, N, G, P);
         const int64_t active = std::min<int64_t>(tiles, sms);
         const int64_t waves = (tiles + sms - 1) / sms;
         const double kpad = (double)((K + BK - 1) / BK * BK);
@@ -413,6 +464,64 @@ int select_tile(int M, int N, int K, int sms) {
         }
     }
     return best;
+}
+
+int select_tile(int M, int N, int K, int sms) { return select_tile_grouped(M, N, K, 1, sms); }
+
+// Validate, encode the tensor maps and launch one grouped GEMM.
+template <int MAXG>
+mr_status launch(const void *A, int64_t lda, const void *const *Wts, int64_t ldw, void *const *Cs, int64_t ldc,
+                 int32_t M, int32_t N, int32_t K, int32_t G, int32_t in_dtype, int32_t out_dtype, int32_t tile_id,
+                 void *stream) {
+    if (!A || !Wts || !Cs) return MR_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < 1 || G < 1 || G > MAXG) return MR_ERR_INVALID_ARG;
+    if (lda < K || ldw < K || ldc < N) return MR_ERR_INVALID_ARG;
+    if (in_dtype != MR_F16 && in_dtype != MR_BF16) return MR_ERR_INVALID_ARG;
+    if (out_dtype != MR_F16 && out_dtype != MR_BF16 && out_dtype != MR_F32) return MR_ERR_INVALID_ARG;
+    if (tile_id < -1 || tile_id >= kNumTiles) return MR_ERR_INVALID_ARG;
+    for (int g = 0; g < G; ++g)
+        if (!Wts[g] || !Cs[g]) return MR_ERR_INVALID_ARG;
+    if (K % 8 != 0 || lda % 8 != 0 || ldw % 8 != 0 || ldc % 8 != 0) return MR_ERR_MISALIGNED;
+    if ((uintptr_t)A & 15u) return MR_ERR_MISALIGNED;
+    for (int g = 0; g < G; ++g)
+        if (((uintptr_t)Wts[g] & 15u) || ((uintptr_t)Cs[g] & 15u)) return MR_ERR_MISALIGNED;
+
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) return mr_host::cuda_status(e);
+    e = init_device(device);
+    if (e != cudaSuccess) return MR_ERR_CUDA;
+    const int sms = mr_host::sm_count() > 0 ? mr_host::sm_count() : 148;
+    const int t = tile_id >= 0 ? tile_id : select_tile_grouped(M, N, K, G, sms);
+    if (t < 0) return MR_ERR_INVALID_ARG;
+    const TileDesc &td = kTiles[t];
+
+    GemmArgs<MAXG> args;
+    memset(&args, 0, sizeof(args));
+    args.P = pack_factor(td.bn, N, G);
+    args.tn_per_group = (N + td.bn - 1) / td.bn;
+    args.ntn = (int)n_slots(td.bn, N, G, args.P);
+    args.M = M;
+    args.N = N;
+    args.K = K;
+    args.G = G;
+    args.ldc = ldc;
+    args.idesc = make_idesc(in_dtype, td.bn);
+    if (!encode_operand(&args.tmA, A, M, K, lda, in_dtype, BM)) return MR_ERR_CUDA;
+    const int b_rows = args.P > 1 ? N : td.bn;
+    for (int g = 0; g < G; ++g) {
+        if (!encode_operand(&args.tmB[g], Wts[g], N, K, ldw, in_dtype, b_rows)) return MR_ERR_CUDA;
+        args.C[g] = Cs[g];
+    }
+
+    const int64_t ntiles = (int64_t)args.ntn * ((M + BM - 1) / BM);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min<int64_t>(ntiles, sms));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem_bytes_for(td.bn, td.stages);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    e = cudaLaunchKernelEx(&cfg, kernel_for<MAXG>(t, out_dtype), args);
+    return mr_host::cuda_status(e);
 }
 
 }  // namespace gemm
@@ -434,37 +543,22 @@ extern "C" int32_t gemm_f16_select_tile(int32_t M, int32_t N, int32_t K) {
 extern "C" mr_status gemm_f16(const void *A, int64_t lda, const void *Wt, int64_t ldw, void *C, int64_t ldc,
                               int32_t M, int32_t N, int32_t K, int32_t in_dtype, int32_t out_dtype, int32_t tile_id,
                               void *stream) {
-    using namespace mr::gemm;
-    if (!A || !Wt || !C) return MR_ERR_INVALID_ARG;
-    if (M < 1 || N < 1 || K < 1) return MR_ERR_INVALID_ARG;
-    if (lda < K || ldw < K || ldc < N) return MR_ERR_INVALID_ARG;
-    if (in_dtype != MR_F16 && in_dtype != MR_BF16) return MR_ERR_INVALID_ARG;
-    if (out_dtype != MR_F16 && out_dtype != MR_BF16 && out_dtype != MR_F32) return MR_ERR_INVALID_ARG;
-    if (tile_id < -1 || tile_id >= kNumTiles) return MR_ERR_INVALID_ARG;
-    if (K % 8 != 0 || lda % 8 != 0 || ldw % 8 != 0 || ldc % 8 != 0) return MR_ERR_MISALIGNED;
-    if (((uintptr_t)A & 15u) || ((uintptr_t)Wt & 15u) || ((uintptr_t)C & 15u)) return MR_ERR_MISALIGNED;
+    const void *w[1] = {Wt};
+    void *c[1] = {C};
+    if (!Wt || !C) return MR_ERR_INVALID_ARG;
+    return mr::gemm::launch<1>(A, lda, w, ldw, c, ldc, M, N, K, 1, in_dtype, out_dtype, tile_id, stream);
+}
 
-    int device = 0;
-    cudaError_t e = cudaGetDevice(&device);
-    if (e != cudaSuccess) return mr_host::cuda_status(e);
-    e = init_device(device);
-    if (e != cudaSuccess) return MR_ERR_CUDA;
-    const int sms = mr_host::sm_count();
-    const int t = tile_id >= 0 ? tile_id : select_tile(M, N, K, sms > 0 ? sms : 148);
-    if (t < 0) return MR_ERR_INVALID_ARG;
-    const TileDesc &td = kTiles[t];
+extern "C" mr_status gemm_f16_grouped(const void *A, int64_t lda, const void *const *Wts, int64_t ldw, void *const *Cs,
+                                      int64_t ldc, int32_t M, int32_t N, int32_t K, int32_t G, int32_t in_dtype,
+                                      int32_t out_dtype, int32_t tile_id, void *stream) {
+    if (G > mr::gemm::kMaxGroups) return MR_ERR_UNSUPPORTED;
+    return mr::gemm::launch<mr::gemm::kMaxGroups>(A, lda, Wts, ldw, Cs, ldc, M, N, K, G, in_dtype, out_dtype,
+                                                  tile_id, stream);
+}
 
-    CUtensorMap ta, tb;
-    if (!encode_operand(&ta, A, M, K, lda, in_dtype, BM)) return MR_ERR_CUDA;
-    if (!encode_operand(&tb, Wt, N, K, ldw, in_dtype, td.bn)) return MR_ERR_CUDA;
-
-    cudaLaunchConfig_t cfg = {};
-    const int64_t ntiles = (int64_t)((N + td.bn - 1) / td.bn) * ((M + BM - 1) / BM);
-    cfg.gridDim = dim3((unsigned)std::min<int64_t>(ntiles, sms > 0 ? sms : 148));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem_bytes_for(td.bn, td.stages);
-    cfg.stream = static_cast<cudaStream_t>(stream);
-    e = cudaLaunchKernelEx(&cfg, kernel_for(t, out_dtype), ta, tb, C, ldc, (int)M, (int)N, (int)K,
-                           make_idesc(in_dtype, td.bn));
-    return mr_host::cuda_status(e);
+extern "C" int32_t gemm_f16_grouped_select_tile(int32_t M, int32_t N, int32_t K, int32_t G) {
+    int sms = mr_host::sm_count();
+    if (sms <= 0) sms = 148;
+    return mr::gemm::select_tile_grouped(M, N, K, G, sms);
 }
