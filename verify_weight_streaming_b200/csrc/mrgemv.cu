@@ -495,22 +495,25 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
 
 using KernelFn = void (*)(const Params);
 
-// Columns per group: at most 64 fp32 accumulators per lane (MB x CG).
-template <int MB>
-constexpr int col_group() { return MB <= 8 ? 8 : 4; }
-inline int col_group_rt(int MB) { return MB <= 8 ? 8 : 4; }
+// Columns per group (one ring slot holds one group): at most 64 fp32
+// accumulators per lane (MB x CG), and slots of about 20 KB for long rows, so
+// that a CTA's whole weight block can be in flight at once (8 columns of a
+// 2560-element row would make 40 KB slots and force slot refills).
+inline int col_group_rt(int MB, int k) { return (MB <= 8 && k <= 1536) ? 8 : 4; }
 
 template <bool FUSED>
-KernelFn kernel_for_mb(int MB) {
+KernelFn kernel_for_mb(int MB, int CG) {
     switch (MB) {
-        case 2: return gemv_kernel<2, col_group<2>(), FUSED>;
-        case 4: return gemv_kernel<4, col_group<4>(), FUSED>;
-        case 8: return gemv_kernel<8, col_group<8>(), FUSED>;
-        default: return gemv_kernel<16, col_group<16>(), FUSED>;
+        case 2: return CG == 8 ? gemv_kernel<2, 8, FUSED> : gemv_kernel<2, 4, FUSED>;
+        case 4: return CG == 8 ? gemv_kernel<4, 8, FUSED> : gemv_kernel<4, 4, FUSED>;
+        case 8: return CG == 8 ? gemv_kernel<8, 8, FUSED> : gemv_kernel<8, 4, FUSED>;
+        default: return gemv_kernel<16, 4, FUSED>;
     }
 }
 
-KernelFn kernel_for(int MB, bool fused) { return fused ? kernel_for_mb<true>(MB) : kernel_for_mb<false>(MB); }
+KernelFn kernel_for(int MB, int CG, bool fused) {
+    return fused ? kernel_for_mb<true>(MB, CG) : kernel_for_mb<false>(MB, CG);
+}
 
 // Rows are processed in pairs, so a single row runs in the 2-row kernel with a zero second row.
 int row_bucket(int m) { return m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
@@ -524,10 +527,11 @@ cudaError_t ensure_attributes(int device) {
     const int optin = mr_host::max_smem_optin();
     const int mbs[] = {2, 4, 8, 16};
     for (int mb : mbs)
-        for (int fused = 0; fused < 2; ++fused) {
-            cudaError_t e = cudaFuncSetAttribute(kernel_for(mb, fused != 0),
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-            if (e != cudaSuccess) return e;
+        for (int cg = 4; cg <= 8; cg += 4)
+            for (int fused = 0; fused < 2; ++fused) {
+                cudaError_t e = cudaFuncSetAttribute(kernel_for(mb, cg, fused != 0),
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+                if (e != cudaSuccess) return e;
         }
     if (device >= 0 && device < 64) g_attr_done[device] = true;
     return cudaSuccess;
@@ -556,7 +560,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     if (k % 8 != 0) return MR_ERR_MISALIGNED;
     if (m > kMaxRows) return MR_ERR_UNSUPPORTED;
     pl.MB = row_bucket(m);
-    pl.CG = col_group_rt(pl.MB);
+    pl.CG = col_group_rt(pl.MB, k);
     pl.KW = k_warps(k);
     pl.G = std::min(sms, n);
     const int cols_max = (n + pl.G - 1) / pl.G;
@@ -577,9 +581,11 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     int s_max = slots_for(budget);
     if (s_max < 1) s_max = slots_for((size_t)optin);
     if (s_max < 1) return MR_ERR_UNSUPPORTED;
-    if (s_max < ng_max && s_max < 2 * std::min(cwg0, 2) && budget < (size_t)optin) {
-        // Refills would leave a consumer warp without a second slot: give up
-        // co-residency with the next launch and take the full shared memory.
+    if (s_max < ng_max && budget < (size_t)optin) {
+        // The block does not fit the co-residency budget, so slots would be
+        // refilled (a second DRAM round trip per refill).  Streaming depth
+        // matters more than overlapping the next launch: take the full shared
+        // memory.
         s_max = std::max(s_max, slots_for((size_t)optin));
     }
     if (s_max >= ng_max) {
@@ -686,7 +692,7 @@ mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = (flags & MR_GEMV_PDL) ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kernel_for(pl.MB, fused != nullptr), p);
+    e = cudaLaunchKernelEx(&cfg, kernel_for(pl.MB, pl.CG, fused != nullptr), p);
     return mr_host::cuda_status(e);
 }
 
