@@ -136,26 +136,36 @@ struct Scatter {
     static constexpr int kReplMask = V >= 32 ? 0 : (32 / V) - 1;
 };
 
+// Floats of k-slice partials: [groups][KW][MB x CG] when k is split over warps.
+__host__ __device__ inline size_t red_floats(int KW, int ng_max, int MB, int CG) {
+    return KW > 1 ? (size_t)ng_max * KW * MB * CG : 0;
+}
+
+// Most column groups any CTA of the launch owns.
+__host__ __device__ inline int ng_max_of(int n, int G, int CG) {
+    const int cols_max = (n + G - 1) / G;
+    return (cols_max + CG - 1) / CG;
+}
+
 struct Smem {
     uint16_t *a;          // [MB][k]
     uint8_t *ring;        // S slots
     uint64_t *full;       // [S]
     uint64_t *empty;      // [S]
-    uint64_t *red_full;   // [CWG]
-    uint64_t *red_free;   // [CWG]
     uint64_t *a_full;     // [1]
+    uint64_t *parts_done; // [1] every warp has written its k-slice partials
     uint64_t *cta_done;   // [1] every warp's logits are stored (fused router)
     uint64_t *decided;    // [1] thread 0 knows whether this CTA finished last
     uint32_t *is_last;    // [2]
     uint64_t *staged;     // [1] the last CTA's copy of the logits is complete
-    float *red;           // [CWG][KW][32][VPL]
+    float *red;           // [groups][KW][MB x CG] k-slice partials (KW > 1)
 };
 
 // One column group: NC (power of two) columns of this warp's k-slice.
-template <int MB, int NC, int VPL>
+template <int MB, int NC, int CGMAX>
 __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g, int ncol,
-                                         int col0, int slice, int cw, int it, int lane,
-                                         int q_begin, int q_end, int chunk_groups) {
+                                         int col0, int slice, int lane, int q_begin, int q_end,
+                                         int chunk_groups) {
     const int k = p.k;
     const int slot = g % p.S;
     // Without refills (chunk_groups > 0) group g waits on the barrier of the
@@ -222,61 +232,42 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     ReduceScatter<V, 16>::run(v, lane, base);
     constexpr int PL = Scatter<V>::kPerLane;
 
-    bool ok = true;
-    if (p.KW > 1) {
-        float *red = sm.red + (size_t)cw * p.KW * 32 * VPL;
-        const uint32_t rpar = (uint32_t)it & 1u;
-        if (slice > 0) {
-            // Wait until slice 0 has consumed the previous group's partials.
-            if (it > 0)
-                ok = mbar_wait_bounded(smem_u32(&sm.red_free[cw]), rpar ^ 1u, MR_DEVERR_GEMV_TIMEOUT);
-            if (ok) {
+    if ((lane & Scatter<V>::kReplMask) == 0) {
+        if (p.KW > 1) {
+            // Partials of this k-slice for group g; the slices are summed, in
+            // slice order, after every group of the CTA is done.
+            float *red = sm.red + ((size_t)g * p.KW + slice) * (MB * CGMAX);
 #pragma unroll
-                for (int i = 0; i < PL; ++i) red[((size_t)slice * 32 + lane) * VPL + i] = v[i];
-                mbar_arrive(smem_u32(&sm.red_full[cw]));
+            for (int i = 0; i < PL; ++i) {
+                const int idx = base + i;
+                red[(idx / NC) * CGMAX + idx % NC] = v[i];
             }
         } else {
-            ok = mbar_wait_bounded(smem_u32(&sm.red_full[cw]), rpar, MR_DEVERR_GEMV_TIMEOUT);
-            if (ok) {
-                for (int s = 1; s < p.KW; ++s)
 #pragma unroll
-                    for (int i = 0; i < PL; ++i)
-                        v[i] = __fadd_rn(v[i], red[((size_t)s * 32 + lane) * VPL + i]);
-                mbar_arrive(smem_u32(&sm.red_free[cw]));
+            for (int i = 0; i < PL; ++i) {
+                const int idx = base + i;
+                const int r = idx / NC, j = idx % NC;
+                if (r < p.m && j < ncol) p.C[(int64_t)r * p.ldc + col0 + j] = v[i];
             }
         }
     }
-
-    if (ok && slice == 0 && (lane & Scatter<V>::kReplMask) == 0) {
-#pragma unroll
-        for (int i = 0; i < PL; ++i) {
-            const int idx = base + i;
-            const int r = idx / NC, j = idx % NC;
-            if (r < p.m && j < ncol) p.C[(int64_t)r * p.ldc + col0 + j] = v[i];
-        }
-    }
-    return ok;
+    return true;
 }
 
-// Run a group of `ncol` valid columns with the smallest power-of-two width
-// NC >= ncol (extra columns compute on whatever the slot holds and are never
-// stored; every column's arithmetic is independent of NC).
-template <int MB, int NC, int VPL>
+template <int MB, int NC, int CGMAX>
 __device__ __forceinline__ bool run_group(const Params &p, const Smem &sm, int g, int ncol,
-                                          int col0, int slice, int cw, int it, int lane,
-                                          int q_begin, int q_end, int chunk_groups) {
+                                          int col0, int slice, int lane, int q_begin, int q_end,
+                                          int chunk_groups) {
     if constexpr (NC > 1) {
         if (ncol <= NC / 2)
-            return run_group<MB, NC / 2, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end,
-                                              chunk_groups);
+            return run_group<MB, NC / 2, CGMAX>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups);
     }
-    return do_group<MB, NC, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end, chunk_groups);
+    return do_group<MB, NC, CGMAX>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups);
 }
 
 template <int MB, int CG, bool FUSED>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    constexpr int VPL = Scatter<MB * CG>::kPerLane;
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -294,13 +285,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     sm.ring = smem_raw + p.a_bytes;
     sm.full = reinterpret_cast<uint64_t *>(sm.ring + (size_t)p.S * p.slot_bytes);
     sm.empty = sm.full + p.S;
-    sm.red_full = sm.empty + p.S;
-    sm.red_free = sm.red_full + p.CWG;
-    sm.a_full = sm.red_free + p.CWG;
+    sm.a_full = sm.empty + p.S;
     sm.cta_done = sm.a_full + 1;
     sm.decided = sm.a_full + 2;
     sm.is_last = reinterpret_cast<uint32_t *>(sm.a_full + 3);
     sm.staged = sm.a_full + 4;
+    sm.parts_done = sm.a_full + 5;
     sm.red = reinterpret_cast<float *>(sm.a_full + 6);
 
     // Groups per copy chunk when no slot is refilled (0 when slots are refilled).
@@ -328,16 +318,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             mbar_init(smem_u32(&sm.empty[s]), (uint32_t)p.KW);
         }
         mbar_init(smem_u32(sm.a_full), 1);
+        mbar_init(smem_u32(sm.parts_done), (uint32_t)(blockDim.x / 32));
         if constexpr (FUSED) {
             mbar_init(smem_u32(sm.cta_done), (uint32_t)(blockDim.x / 32));
             mbar_init(smem_u32(sm.decided), 1);
             mbar_init(smem_u32(sm.staged), 1);
-        }
-        if (p.KW > 1) {
-            for (int c = 0; c < p.CWG; ++c) {
-                mbar_init(smem_u32(&sm.red_full[c]), (uint32_t)(p.KW - 1) * 32u);
-                mbar_init(smem_u32(&sm.red_free[c]), 32u);
-            }
         }
         fence_mbar_init();
         if (ng <= p.S) {
@@ -394,11 +379,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     const int q_begin = (int)(((int64_t)slice * q_total) / p.KW);
     const int q_end = (int)(((int64_t)(slice + 1) * q_total) / p.KW);
 
-    int it = 0;
-    for (int g = cw; g < ng && !failed; g += p.CWG, ++it) {
+    for (int g = cw; g < ng && !failed; g += p.CWG) {
         const int col0 = c_begin + g * CG;
         const int ncol = min(CG, c_end - col0);
-        if (!run_group<MB, CG, VPL>(p, sm, g, ncol, col0, slice, cw, it, lane, q_begin, q_end, chunk_groups)) {
+        if (!run_group<MB, CG, CG>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups)) {
             failed = true;
             break;
         }
@@ -415,6 +399,25 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             }
             if (lane == 0) issue_group(g + p.S);
             __syncwarp();
+        }
+    }
+
+    if (p.KW > 1) {
+        // Sum the k-slices of every output in slice order and store C; one
+        // barrier for the CTA instead of one handshake per group.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(sm.parts_done));
+        if (!mbar_wait_bounded(smem_u32(sm.parts_done), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
+        constexpr int VCG = MB * CG;
+        for (int e = tid; e < ng * VCG; e += blockDim.x) {
+            const int g = e / VCG, rem = e % VCG;
+            const int r = rem / CG, col = c_begin + g * CG + rem % CG;
+            if (r < p.m && col < c_end) {
+                const float *src = sm.red + (size_t)g * p.KW * VCG + rem;
+                float acc = src[0];
+                for (int sl = 1; sl < p.KW; ++sl) acc = __fadd_rn(acc, src[(size_t)sl * VCG]);
+                p.C[(int64_t)r * p.ldc + col] = acc;
+            }
         }
     }
 
@@ -478,7 +481,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             }
             if (!mbar_wait_bounded(smem_u32(sm.staged), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
         }
-        uint64_t *tk = reinterpret_cast<uint64_t *>(sm.red + (size_t)p.CWG * p.KW * 32 * VPL) + warp * 64;
+        uint64_t *tk = reinterpret_cast<uint64_t *>(sm.red + red_floats(p.KW, ng_max_of(p.n, p.G, CG), MB, CG)) + warp * 64;
         for (int r = warp; r < p.m; r += nwarps) {
             const float *x = staged ? lg + (size_t)r * p.n : p.C + (int64_t)r * p.ldc;
             const uint64_t best = topk::warp_topk_fast<16>(x, p.n, p.topk, lane, 0, 1, 0ull, tk);
@@ -563,15 +566,13 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     pl.CG = col_group_rt(pl.MB, k);
     pl.KW = k_warps(k);
     pl.G = std::min(sms, n);
-    const int cols_max = (n + pl.G - 1) / pl.G;
-    const int ng_max = (cols_max + pl.CG - 1) / pl.CG;
+    const int ng_max = ng_max_of(n, pl.G, pl.CG);
     const int cwg0 = std::max(1, std::min(ng_max, kMaxWarps / pl.KW));
     pl.a_bytes = (uint32_t)(((size_t)pl.MB * k * 2 + 127) / 128 * 128);
     pl.slot_bytes = (uint32_t)pl.CG * (uint32_t)k * 2u;
-    const size_t vpl = (size_t)std::max(1, pl.MB * pl.CG / 32);
+    const size_t red_bytes = red_floats(pl.KW, ng_max, pl.MB, pl.CG) * sizeof(float);
     const size_t topk_bytes = fused ? (size_t)kMaxWarps * 64 * 8 : 0;
-    const size_t fixed = topk_bytes + pl.a_bytes + 16 * (size_t)(2 * ng_max + 2 * cwg0) + 48 +
-                         (size_t)cwg0 * pl.KW * 32 * vpl * 4 + 64;
+    const size_t fixed = topk_bytes + pl.a_bytes + 16 * (size_t)ng_max + 48 + red_bytes + 64;
     const size_t pdl_budget = 110 * 1024;
     const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, (size_t)optin) : (size_t)optin;
     auto slots_for = [&](size_t b) -> int {
@@ -596,8 +597,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
         pl.CWG = std::max(1, std::min(cwg0, s_max / 2));
         pl.S = (s_max / pl.CWG) * pl.CWG;
     }
-    pl.smem = topk_bytes + pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 16 * (size_t)(pl.S + pl.CWG) + 48 +
-              (size_t)pl.CWG * pl.KW * 32 * vpl * 4;
+    pl.smem = topk_bytes + pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 16 * (size_t)pl.S + 48 + red_bytes;
     if (pl.smem > (size_t)optin) return MR_ERR_UNSUPPORTED;
     return MR_OK;
 }
