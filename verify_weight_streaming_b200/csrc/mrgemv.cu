@@ -150,7 +150,8 @@ __host__ __device__ inline int ng_max_of(int n, int G, int CG) {
 struct Smem {
     uint16_t *a;          // [MB][k]
     uint8_t *ring;        // S slots
-    uint64_t *full;       // [S]
+    uint64_t *chunk_full; // [S] first pass: one barrier per up-front copy chunk
+    uint64_t *full;       // [S] refills: slot s's uses 1, 2, ...
     uint64_t *empty;      // [S]
     uint64_t *a_full;     // [1]
     uint64_t *parts_done; // [1] every warp has written its k-slice partials
@@ -168,12 +169,12 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
                                          int chunk_groups) {
     const int k = p.k;
     const int slot = g % p.S;
-    // Without refills (chunk_groups > 0) group g waits on the barrier of the
-    // copy chunk that holds it, phase 0; with refills, on its slot's barrier
-    // for use g / S.
-    const int bar_idx = chunk_groups > 0 ? g / chunk_groups : slot;
-    const uint32_t par = chunk_groups > 0 ? 0u : (uint32_t)(g / p.S) & 1u;
-    if (!mbar_wait_bounded(smem_u32(&sm.full[bar_idx]), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
+    // The first S groups come in up-front copy chunks (one barrier each,
+    // phase 0); group g >= S is the refill of its slot, use g / S, counted on
+    // the slot's refill barrier from phase 0.
+    const uint64_t *bar = g < p.S ? &sm.chunk_full[g / chunk_groups] : &sm.full[slot];
+    const uint32_t par = g < p.S ? 0u : (uint32_t)(g / p.S - 1) & 1u;
+    if (!mbar_wait_bounded(smem_u32(bar), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
 
     const uint32_t w_s = smem_u32(sm.ring + (size_t)slot * p.slot_bytes);
     const uint32_t a_s = smem_u32(sm.a);
@@ -283,7 +284,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     Smem sm;
     sm.a = reinterpret_cast<uint16_t *>(smem_raw);
     sm.ring = smem_raw + p.a_bytes;
-    sm.full = reinterpret_cast<uint64_t *>(sm.ring + (size_t)p.S * p.slot_bytes);
+    sm.chunk_full = reinterpret_cast<uint64_t *>(sm.ring + (size_t)p.S * p.slot_bytes);
+    sm.full = sm.chunk_full + p.S;
     sm.empty = sm.full + p.S;
     sm.a_full = sm.empty + p.S;
     sm.cta_done = sm.a_full + 1;
@@ -294,7 +296,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     sm.red = reinterpret_cast<float *>(sm.a_full + 6);
 
     // Groups per copy chunk when no slot is refilled (0 when slots are refilled).
-    const int chunk_groups = ng <= p.S ? (int)max(1u, (32768u + p.slot_bytes - 1) / p.slot_bytes) : 0;
+    const int chunk_groups = (int)max(1u, (32768u + p.slot_bytes - 1) / p.slot_bytes);
+    const int first = min(ng, p.S);
 
     auto issue_group = [&](int g) {
         const int slot = g % p.S;
@@ -314,6 +317,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
 
     if (tid == 0) {
         for (int s = 0; s < p.S; ++s) {
+            mbar_init(smem_u32(&sm.chunk_full[s]), 1);
             mbar_init(smem_u32(&sm.full[s]), 1);
             mbar_init(smem_u32(&sm.empty[s]), (uint32_t)p.KW);
         }
@@ -325,27 +329,24 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             mbar_init(smem_u32(sm.staged), 1);
         }
         fence_mbar_init();
-        if (ng <= p.S) {
-            // Everything fits: copy in chunks of whole groups of >= 32 KB each
-            // (small bulk copies stream below HBM bandwidth: ~2.6 TB/s for
-            // 4 KB copies, ~6.2 TB/s for 16 KB, ~7 TB/s for 32-64 KB).
-            const uint32_t row_bytes = (uint32_t)k * 2u;
-            for (int c = 0; c * chunk_groups < ng; ++c) {
-                const int g0 = c * chunk_groups;
-                const int cc0 = c_begin + g0 * CG;
-                const int nc = min(chunk_groups * CG, c_end - cc0);
-                const uint32_t bar = smem_u32(&sm.full[c]);
-                const uint32_t dst = smem_u32(sm.ring + (size_t)g0 * p.slot_bytes);
-                mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)nc);
-                if (p.ldw == k) {
-                    bulk_g2s(dst, p.Wt + (int64_t)cc0 * k, row_bytes * (uint32_t)nc, bar);
-                } else {
-                    for (int j = 0; j < nc; ++j)
-                        bulk_g2s(dst + j * row_bytes, p.Wt + (int64_t)(cc0 + j) * p.ldw, row_bytes, bar);
-                }
+        // The first min(ng, S) groups: copy in chunks of whole groups of
+        // >= 32 KB each (small bulk copies stream below HBM bandwidth: ~2.6
+        // TB/s for 4 KB copies, ~6.2 TB/s for 16 KB, ~7 TB/s for 32-64 KB).
+        const uint32_t row_bytes = (uint32_t)k * 2u;
+        for (int c = 0; c * chunk_groups < first; ++c) {
+            const int g0 = c * chunk_groups;
+            const int g1 = min(g0 + chunk_groups, first);
+            const int cc0 = c_begin + g0 * CG;
+            const int nc = min((g1 - g0) * CG, c_end - cc0);
+            const uint32_t bar = smem_u32(&sm.chunk_full[c]);
+            const uint32_t dst = smem_u32(sm.ring + (size_t)g0 * p.slot_bytes);
+            mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)nc);
+            if (p.ldw == k) {
+                bulk_g2s(dst, p.Wt + (int64_t)cc0 * k, row_bytes * (uint32_t)nc, bar);
+            } else {
+                for (int j = 0; j < nc; ++j)
+                    bulk_g2s(dst + j * row_bytes, p.Wt + (int64_t)(cc0 + j) * p.ldw, row_bytes, bar);
             }
-        } else {
-            for (int g = 0; g < p.S; ++g) issue_group(g);
         }
     }
     // The weight stream is in flight; the next kernel may start launching.
@@ -573,7 +574,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     pl.slot_bytes = (uint32_t)pl.CG * (uint32_t)k * 2u;
     const size_t red_bytes = red_floats(pl.KW, ng_max, pl.MB, pl.CG) * sizeof(float);
     const size_t topk_bytes = fused ? (size_t)kMaxWarps * 64 * 8 : 0;
-    const size_t fixed = topk_bytes + pl.a_bytes + 16 * (size_t)ng_max + 48 + red_bytes + 64;
+    const size_t fixed = topk_bytes + pl.a_bytes + 24 * (size_t)ng_max + 48 + red_bytes + 64;
     const size_t pdl_budget = 110 * 1024;
     const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, (size_t)optin) : (size_t)optin;
     auto slots_for = [&](size_t b) -> int {
@@ -598,7 +599,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
         pl.CWG = std::max(1, std::min(cwg0, s_max / 2));
         pl.S = (s_max / pl.CWG) * pl.CWG;
     }
-    pl.smem = topk_bytes + pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 16 * (size_t)pl.S + 48 + red_bytes;
+    pl.smem = topk_bytes + pl.a_bytes + (size_t)pl.S * pl.slot_bytes + 24 * (size_t)pl.S + 48 + red_bytes;
     if (pl.smem > (size_t)optin) return MR_ERR_UNSUPPORTED;
     return MR_OK;
 }
