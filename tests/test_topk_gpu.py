@@ -57,7 +57,7 @@ def test_router_window_on_gpu_logits(m):
 
 
 @pytest.mark.parametrize("n,k", [(512, 10), (1, 1), (7, 7), (31, 10), (128, 32), (129, 1),
-                                 (1000, 17), (5000, 10), (4097, 32)])
+                                 (1000, 17), (2048, 32), (2049, 10), (5000, 10), (4097, 32)])
 def test_shapes(n, k):
     x = synth.bits_to_float32(synth.normal_bits(400 + n, (6, n), "bf16", 1.0), "bf16")
     check(x, k)

@@ -15,7 +15,7 @@
 // pass (k rounds of a warp-wide maximum when ties leave more than 32).  The
 // CTA's warps are merged the same way at the end.  Values are re-read from
 // the logits at the selected indices so they match bit for bit (a -0.0 stays
-// -0.0).
+// -0.0).  Rows of up to 2048 logits take one warp per row instead.
 #include "common.cuh"
 
 #include "topk_core.cuh"
@@ -57,6 +57,26 @@ __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float *__restri
     }
 }
 
+// Rows of up to kWarpRowMax logits: one warp per row (a 32-thread CTA),
+// chunks of 512 elements, no cross-warp merge and no block barrier.
+constexpr int kWarpRowMax = 2048;
+
+__global__ void __launch_bounds__(32) topk_warp_kernel(const float *__restrict__ logits, int64_t ldl, int n, int K,
+                                                       int32_t *__restrict__ idx, float *__restrict__ val,
+                                                       int64_t ldo) {
+    __shared__ uint64_t scratch[64];
+    const int lane = threadIdx.x;
+    const int64_t row = blockIdx.x;
+    const float *x = logits + row * ldl;
+    grid_launch_dependents();
+    grid_dependency_wait();
+    const uint64_t best = warp_topk_fast<16>(x, n, K, lane, 0, 1, 0ull, scratch);
+    if (lane < K) {
+        idx[row * ldo + lane] = (int32_t)key_index(best);
+        if (val) val[row * ldo + lane] = selected_value(best, x);
+    }
+}
+
 }  // namespace topk
 }  // namespace mr
 
@@ -67,9 +87,10 @@ extern "C" mr_status router_topk(const float *logits, int64_t ldl, int32_t m, in
     if (ldl < n || ldo < topk) return MR_ERR_INVALID_ARG;
     if (topk > mr::topk::kMaxK) return MR_ERR_UNSUPPORTED;
     if (((uintptr_t)logits & 3u) || ((uintptr_t)idx & 3u) || ((uintptr_t)val & 3u)) return MR_ERR_MISALIGNED;
+    const bool one_warp = n <= mr::topk::kWarpRowMax;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)m);
-    cfg.blockDim = dim3(mr::topk::kWarps * 32);
+    cfg.blockDim = dim3(one_warp ? 32 : mr::topk::kWarps * 32);
     cfg.stream = static_cast<cudaStream_t>(stream);
     // Safe for any predecessor: the kernel waits for it before reading input.
     cudaLaunchAttribute attr[1];
@@ -77,6 +98,9 @@ extern "C" mr_status router_topk(const float *logits, int64_t ldl, int32_t m, in
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (one_warp)
+        return mr_host::cuda_status(
+            cudaLaunchKernelEx(&cfg, mr::topk::topk_warp_kernel, logits, ldl, (int)n, (int)topk, idx, val, ldo));
     return mr_host::cuda_status(
         cudaLaunchKernelEx(&cfg, mr::topk::topk_kernel, logits, ldl, (int)n, (int)topk, idx, val, ldo));
 }
