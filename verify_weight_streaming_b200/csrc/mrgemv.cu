@@ -17,10 +17,10 @@
 //    the slot's successive uses in order.  The first slots are
 //    requested before griddepcontrol.wait, so under programmatic dependent
 //    launch the weight stream overlaps the previous kernel.
-//  * A (m rows, bf16) is staged once in shared memory by per-thread cp.async
-//    copies issued after the grid-dependency wait (the bulk-copy engine would
-//    serve it only after the weight copies issued before); rows m..MB-1 are
-//    zero.
+//  * A (m rows, bf16) is staged once in shared memory by a bulk copy issued
+//    after the grid-dependency wait, right after the first weight chunk and
+//    before the others (copies from one CTA are served roughly in order, so A
+//    must not queue behind the whole weight block); rows m..MB-1 are zero.
 //  * Lanes split k in 4-element chunks: chunk q belongs to lane q % 32 of the
 //    k-slice that holds it.  KW warps split k into contiguous slices; KW is a
 //    function of k alone.  Each lane keeps one fp32 accumulator per (row,
@@ -155,7 +155,7 @@ struct Smem {
     uint64_t *chunk_full; // [S] first pass: one barrier per up-front copy chunk
     uint64_t *full;       // [S] refills: slot s's uses 1, 2, ...
     uint64_t *empty;      // [S]
-    uint64_t *a_full;     // [1] (unused slot; keeps the barrier block layout)
+    uint64_t *a_full;     // [1] A has landed
     uint64_t *parts_done; // [1] every warp has written its k-slice partials
     uint64_t *cta_done;   // [1] every warp's logits are stored (fused router)
     uint64_t *decided;    // [1] thread 0 knows whether this CTA finished last
@@ -301,6 +301,23 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
     const int chunk_groups = (int)max(1u, (32768u + p.slot_bytes - 1) / p.slot_bytes);
     const int first = min(ng, p.S);
 
+    auto issue_chunk = [&](int c) {
+        const uint32_t row_bytes = (uint32_t)k * 2u;
+        const int g0 = c * chunk_groups;
+        const int g1 = min(g0 + chunk_groups, first);
+        const int cc0 = c_begin + g0 * CG;
+        const int nc = min((g1 - g0) * CG, c_end - cc0);
+        const uint32_t bar = smem_u32(&sm.chunk_full[c]);
+        const uint32_t dst = smem_u32(sm.ring + (size_t)g0 * p.slot_bytes);
+        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)nc);
+        if (p.ldw == k) {
+            bulk_g2s(dst, p.Wt + (int64_t)cc0 * k, row_bytes * (uint32_t)nc, bar);
+        } else {
+            for (int j = 0; j < nc; ++j)
+                bulk_g2s(dst + j * row_bytes, p.Wt + (int64_t)(cc0 + j) * p.ldw, row_bytes, bar);
+        }
+    };
+
     auto issue_group = [&](int g) {
         const int slot = g % p.S;
         const int gc0 = c_begin + g * CG;
@@ -323,6 +340,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             mbar_init(smem_u32(&sm.full[s]), 1);
             mbar_init(smem_u32(&sm.empty[s]), (uint32_t)p.KW);
         }
+        mbar_init(smem_u32(sm.a_full), 1);
         mbar_init(smem_u32(sm.parts_done), (uint32_t)(blockDim.x / 32));
         if constexpr (FUSED) {
             mbar_init(smem_u32(sm.cta_done), (uint32_t)(blockDim.x / 32));
@@ -330,52 +348,41 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
             mbar_init(smem_u32(sm.staged), 1);
         }
         fence_mbar_init();
-        // The first min(ng, S) groups: copy in chunks of whole groups of
+        // The first min(ng, S) groups come in chunks of whole groups of
         // >= 32 KB each (small bulk copies stream below HBM bandwidth: ~2.6
         // TB/s for 4 KB copies, ~6.2 TB/s for 16 KB, ~7 TB/s for 32-64 KB).
-        const uint32_t row_bytes = (uint32_t)k * 2u;
-        for (int c = 0; c * chunk_groups < first; ++c) {
-            const int g0 = c * chunk_groups;
-            const int g1 = min(g0 + chunk_groups, first);
-            const int cc0 = c_begin + g0 * CG;
-            const int nc = min((g1 - g0) * CG, c_end - cc0);
-            const uint32_t bar = smem_u32(&sm.chunk_full[c]);
-            const uint32_t dst = smem_u32(sm.ring + (size_t)g0 * p.slot_bytes);
-            mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)nc);
-            if (p.ldw == k) {
-                bulk_g2s(dst, p.Wt + (int64_t)cc0 * k, row_bytes * (uint32_t)nc, bar);
-            } else {
-                for (int j = 0; j < nc; ++j)
-                    bulk_g2s(dst + j * row_bytes, p.Wt + (int64_t)(cc0 + j) * p.ldw, row_bytes, bar);
-            }
-        }
+        // Chunk 0 is requested now, before the wait for the previous kernel.
+        issue_chunk(0);
     }
     // The weight stream is in flight; the next kernel may start launching.
     grid_launch_dependents();
     // A may be produced by the previous kernel on the stream.
     grid_dependency_wait();
 
-    // Stage A (bf16) in shared memory; rows m..MB-1 are zero.  Every thread
-    // issues 16-byte cp.async copies (not the bulk-copy engine, where A would
-    // queue behind the weight copies issued above), then waits for its own
-    // copies; the CTA barrier makes all of them visible.
+    // Stage A (bf16) in shared memory with one bulk copy (per row if strided);
+    // rows m..MB-1 are zero.  Only the first weight chunk was requested
+    // before this point, so A does not queue behind the whole weight stream;
+    // the remaining chunks follow it.
+    if (tid == 0) {
+        const uint32_t row_bytes = (uint32_t)k * 2u;
+        const uint32_t bar = smem_u32(sm.a_full);
+        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)p.m);
+        if (p.lda == k) {
+            bulk_g2s(smem_u32(sm.a), p.A, row_bytes * (uint32_t)p.m, bar);
+        } else {
+            for (int r = 0; r < p.m; ++r)
+                bulk_g2s(smem_u32(sm.a + (size_t)r * k), p.A + (int64_t)r * p.lda, row_bytes, bar);
+        }
+        for (int c = 1; c * chunk_groups < first; ++c) issue_chunk(c);
+    }
     {
         const int chunks = k / 8;  // 16-byte chunks per row
-        const uint32_t a_s = smem_u32(sm.a);
-        for (int e = tid; e < p.m * chunks; e += blockDim.x) {
-            const int r = e / chunks, c = e % chunks;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
-                         ::"r"(a_s + (uint32_t)(r * k + 8 * c) * 2u), "l"(p.A + (int64_t)r * p.lda + 8 * c)
-                         : "memory");
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
         for (int e = p.m * chunks + tid; e < MB * chunks; e += blockDim.x)
             *reinterpret_cast<uint4 *>(sm.a + (size_t)(e / chunks) * k + 8 * (e % chunks)) =
                 make_uint4(0u, 0u, 0u, 0u);
-        asm volatile("cp.async.wait_all;" ::: "memory");
     }
     __syncthreads();
-    bool failed = false;
+    bool failed = !mbar_wait_bounded(smem_u32(sm.a_full), 0u, MR_DEVERR_GEMV_TIMEOUT);
 
     const int slice = warp % p.KW;
     const int cw = warp / p.KW;
