@@ -70,6 +70,11 @@ class Oracle:
         L.oracle_ulp_bf16.argtypes = [ctypes.c_double]
         L.oracle_ulp_bf16.restype = ctypes.c_double
         L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
+        L.oracle_f32_to_bf16.restype = ctypes.c_uint16
+        L.oracle_cast_f32_bf16.argtypes = [P, I64, P, I64, I64, I64]
+        L.oracle_sigmoid.argtypes = [ctypes.c_double]
+        L.oracle_sigmoid.restype = ctypes.c_double
         self.L = L
 
     def dec_bf16(self, h: int) -> float:
@@ -115,6 +120,21 @@ class Oracle:
     def num_threads(self) -> int:
         return int(self.L.oracle_num_threads())
 
+    def f32_to_bf16(self, x: float) -> int:
+        return int(self.L.oracle_f32_to_bf16(float(x)))
+
+    def cast_f32_bf16(self, x: np.ndarray) -> np.ndarray:
+        """fp32 rows -> bf16 bit patterns (round to nearest even)."""
+        x = np.ascontiguousarray(x, dtype=np.float32)
+        rows, cols = x.shape
+        y = np.empty((rows, cols), dtype=np.uint16)
+        self.L.oracle_cast_f32_bf16(_ptr(x), cols, _ptr(y), cols, rows, cols)
+        return y
+
+    def sigmoid(self, x) -> np.ndarray:
+        flat = np.asarray(x, dtype=np.float64).ravel()
+        return np.array([self.L.oracle_sigmoid(float(v)) for v in flat]).reshape(np.shape(x))
+
 
 _default = None
 
@@ -148,6 +168,22 @@ def ulp(x, fmt):
 
 def num_threads() -> int:
     return default().num_threads()
+
+
+def cast_f32_bf16(x):
+    return default().cast_f32_bf16(x)
+
+
+def sigmoid(x):
+    return default().sigmoid(x)
+
+
+def gate_tolerance(c64: np.ndarray, s64: np.ndarray) -> np.ndarray:
+    """Allowance for sigmoid(C): the GEMV's 1e-5*S through the sigmoid's
+    slope (never above 1/4), plus 4 fp32 ulps of the result for the rounding of
+    exp, the add and the divide."""
+    sig = sigmoid(c64)
+    return 0.25 * REL_TOL * s64 + 4.0 * np.spacing(np.abs(sig).astype(np.float32)).astype(np.float64)
 
 
 def ulp_vec(x: np.ndarray, fmt: str) -> np.ndarray:

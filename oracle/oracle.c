@@ -195,3 +195,37 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* ---- bf16 cast and sigmoid gate (adjacent window steps) ------------------ */
+
+/*
+ * fp32 -> bf16 with round to nearest, ties to even, from the binary32 bit
+ * layout: keep the top 16 bits and round on the 16 dropped ones.  NaN maps to
+ * a quiet NaN of the same sign; overflow rounds to infinity like any other
+ * carry into the exponent field.  (The bf16 cast of the window's rows in
+ * Strata PR #109, "What": one call casts the window's contiguous rows.)
+ */
+uint16_t oracle_f32_to_bf16(float x)
+{
+    uint32_t b;
+    memcpy(&b, &x, sizeof(b));
+    if ((b & 0x7F800000u) == 0x7F800000u && (b & 0x007FFFFFu))
+        return (uint16_t)((b >> 16) | 0x0040u);          /* quiet NaN */
+    uint32_t upper = b >> 16, lower = b & 0xFFFFu;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))
+        upper += 1u;                                      /* carries may reach the exponent */
+    return (uint16_t)upper;
+}
+
+void oracle_cast_f32_bf16(const float *x, int64_t ldx, uint16_t *y, int64_t ldy, int64_t rows, int64_t cols)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            y[r * ldy + c] = oracle_f32_to_bf16(x[r * ldx + c]);
+}
+
+/* The logistic function 1 / (1 + e^-x) in fp64 (the shared expert's scalar gate). */
+double oracle_sigmoid(double x)
+{
+    return 1.0 / (1.0 + exp(-x));
+}

@@ -27,6 +27,9 @@ MUTANTS = {
     "nan_ranked_last": ("return xn ? -1 : 1;", "return xn ? 1 : -1;"),
     "ulp_f16_fraction_bits": ("(e - 1) - 10)", "(e - 1) - 11)"),
     "ulp_bf16_binade": ("(e - 1) - 7)", "e - 7)"),
+    "bf16_ties_away": ("lower > 0x8000u || (lower == 0x8000u && (upper & 1u))", "lower >= 0x8000u"),
+    "bf16_truncate": ("upper += 1u;", "upper += 0u;"),
+    "sigmoid_sign": ("1.0 / (1.0 + exp(-x))", "1.0 / (1.0 + exp(x))"),
 }
 
 

@@ -204,10 +204,49 @@ def pin_ulp(orc):
     assert np.array_equal(got, np.array(list(hand.values())))
 
 
+def pin_cast_bf16(orc):
+    """fp32 -> bf16 round to nearest even, checked against exact fp64 arithmetic."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    with np.errstate(invalid="ignore"):
+        vals = (bits << np.uint32(16)).view(np.float32)
+    finite = np.isfinite(vals)
+    # (a) every bf16 value is its own image
+    got = orc.cast_f32_bf16(vals[finite][None, :])[0]
+    assert np.array_equal(got, bits[finite].astype(np.uint16))
+    # (b) halfway points go to the even neighbour, (c) just off them to the nearer one
+    rng = np.random.default_rng(7)
+    lo = bits[finite & (bits & 0x7FFF < 0x7F7F)][rng.choice(30000, 400, replace=False)]
+    for b in lo:
+        x = float((np.uint32(b) << np.uint32(16)).view(np.float32))
+        nb = int(b) + 1 if x >= 0 else int(b) - 1 if (int(b) & 0x7FFF) else int(b) + 1
+        xn = float((np.uint32(b + 1) << np.uint32(16)).view(np.float32))
+        mid = np.float32((x + xn) / 2.0)          # exact in fp32 (8 more bits)
+        even = b if (b & 1) == 0 else b + 1
+        assert orc.f32_to_bf16(mid) == even, (hex(b), mid)
+        above = np.nextafter(mid, np.float32(np.inf) if xn > x else np.float32(-np.inf))
+        below = np.nextafter(mid, np.float32(-np.inf) if xn > x else np.float32(np.inf))
+        assert orc.f32_to_bf16(above) == b + 1 and orc.f32_to_bf16(below) == b, hex(b)
+    # (d) overflow: half an ulp above the largest finite bf16 rounds to infinity
+    big = (np.uint32(0x7F7F8000)).view(np.float32)
+    assert orc.f32_to_bf16(big) == 0x7F80 and orc.f32_to_bf16(-big) == 0xFF80
+    # (e) NaN stays NaN
+    assert (orc.f32_to_bf16(float("nan")) & 0x7F80) == 0x7F80 and (orc.f32_to_bf16(float("nan")) & 0x7F)
+
+
+def pin_sigmoid(orc):
+    """Closed forms of the logistic function."""
+    x = np.array([0.0, np.log(3.0), -np.log(3.0), np.log(9.0), 40.0, -40.0, 1.5, -2.25])
+    s = orc.sigmoid(x)
+    assert s[0] == 0.5
+    assert abs(s[1] - 0.75) < 1e-15 and abs(s[2] - 0.25) < 1e-15 and abs(s[3] - 0.9) < 1e-15
+    assert 1 - 1e-15 <= s[4] <= 1.0 and 0 < s[5] < 1e-17
+    assert np.all(np.abs(orc.sigmoid(x) + orc.sigmoid(-x) - 1.0) < 1e-15)
+
+
 ALL_PINS = [pin_decode_bf16, pin_decode_f16, pin_integer_bruteforce, pin_mixed_formats,
             pin_worked_example, pin_identity_and_permutation, pin_closed_forms,
             pin_invariants, pin_statistics, pin_topk_bruteforce, pin_topk_library_sort,
-            pin_ulp]
+            pin_ulp, pin_cast_bf16, pin_sigmoid]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
