@@ -61,6 +61,13 @@ enum { MR_F16 = 0, MR_BF16 = 1, MR_F32 = 2 };
 
 /* Flags for mrgemv_bf16_ex. */
 #define MR_GEMV_PDL 0x1u
+#define MR_GEMV_SIGMOID 0x2u
+/*
+ * MR_GEMV_SIGMOID: store 1 / (1 + exp(-c)) for every output c (CUDA's expf,
+ * IEEE division): the shared expert's scalar gate of Strata PR #109 ("What":
+ * one multi-row GEMV with n = 1 plus a sigmoid), here in the same launch.
+ * Not accepted by router_gemv_topk.
+ */
 /*
  * MR_GEMV_PDL: launch with programmatic dependent launch.  The kernel starts
  * streaming its weight into shared memory BEFORE the previous kernel on the
@@ -182,6 +189,19 @@ size_t router_gemv_topk_noalloc_max_logits(void);
 mr_status router_topk(const float *logits, int64_t ldl, int32_t m, int32_t n,
                       int32_t topk, int32_t *idx, float *val, int64_t ldo,
                       void *stream);
+
+/*
+ * cast_f32_bf16 -- fp32 -> bf16, round to nearest even, for `rows` rows of
+ * `cols` values in one launch: the bf16 cast of the verify window's rows in
+ * Strata PR #109 ("What": one call, the rows are contiguous), which feeds the
+ * bf16 A of mrgemv_bf16.  NaN stays NaN; overflow rounds to infinity.
+ *
+ * X : rows x cols fp32, row stride ldx (>= cols) elements, 4-byte aligned.
+ * Y : rows x cols bf16, row stride ldy (>= cols) elements, 2-byte aligned.
+ * Rows of 8k elements with 16-byte aligned rows take a vectorised path.
+ */
+mr_status cast_f32_bf16(const float *X, int64_t ldx, void *Y, int64_t ldy, int32_t rows, int32_t cols,
+                        void *stream);
 
 /*
  * gemm_f16 -- tiled GEMM on the tcgen05 tensor cores (TMA -> shared memory

@@ -48,7 +48,7 @@ def gemv(A=A16, lda=64, W=A16, ldw=64, C=A16, ldc=32, m=4, n=32, k=64, flags=0):
     (dict(C=None), mr.MR_ERR_INVALID_ARG), (dict(m=0), mr.MR_ERR_INVALID_ARG),
     (dict(n=0), mr.MR_ERR_INVALID_ARG), (dict(k=0), mr.MR_ERR_INVALID_ARG),
     (dict(lda=56), mr.MR_ERR_INVALID_ARG), (dict(ldc=31), mr.MR_ERR_INVALID_ARG),
-    (dict(flags=2), mr.MR_ERR_INVALID_ARG),
+    (dict(flags=4), mr.MR_ERR_INVALID_ARG),
     (dict(k=60, lda=64, ldw=64), mr.MR_ERR_MISALIGNED), (dict(lda=68), mr.MR_ERR_MISALIGNED),
     (dict(A=BAD), mr.MR_ERR_MISALIGNED), (dict(W=BAD), mr.MR_ERR_MISALIGNED),
     (dict(m=17), mr.MR_ERR_UNSUPPORTED),
@@ -147,3 +147,23 @@ def test_grouped_validation():
     assert g(A16, 64, Wb, 64, C, 32, 4, 32, 64, 2, 0, 0, -1, None) == mr.MR_ERR_MISALIGNED
     assert g(A16, 64, W, 64, C, 32, 4, 32, 64, 2, 0, 0, -1, None) == mr.MR_ERR_CUDA  # valid; no device
     assert 0 <= mr.gemm_f16_grouped_select_tile(2048, 96, 2560, 36) < mr.gemm_f16_num_tiles()
+
+
+def test_cast_validation():
+    c = mr.lib.cast_f32_bf16
+    assert c(None, 8, A16, 8, 1, 8, None) == mr.MR_ERR_INVALID_ARG
+    assert c(A16, 8, None, 8, 1, 8, None) == mr.MR_ERR_INVALID_ARG
+    assert c(A16, 8, A16, 8, 0, 8, None) == mr.MR_ERR_INVALID_ARG
+    assert c(A16, 4, A16, 8, 1, 8, None) == mr.MR_ERR_INVALID_ARG
+    assert c(P(258), 8, A16, 8, 1, 8, None) == mr.MR_ERR_MISALIGNED
+    assert c(A16, 8, P(257), 8, 1, 8, None) == mr.MR_ERR_MISALIGNED
+    assert c(A16, 8, A16, 8, 1, 8, None) == mr.MR_ERR_CUDA  # valid; no device
+
+
+def test_gate_flag_validation():
+    assert gemv(flags=mr.MR_GEMV_SIGMOID) == mr.MR_ERR_CUDA          # accepted; no device
+    assert gemv(flags=mr.MR_GEMV_SIGMOID | mr.MR_GEMV_PDL) == mr.MR_ERR_CUDA
+    assert gemv(flags=4) == mr.MR_ERR_INVALID_ARG
+    st = mr.lib.router_gemv_topk(A16, 64, A16, 64, None, 512, 4, 512, 64, 10, A16, None, 10, P(512),
+                                 1 << 20, mr.MR_GEMV_SIGMOID, None)
+    assert st == mr.MR_ERR_INVALID_ARG

@@ -17,12 +17,13 @@ from ._build import LIB, build  # noqa: F401
 MR_OK, MR_ERR_INVALID_ARG, MR_ERR_MISALIGNED, MR_ERR_UNSUPPORTED, MR_ERR_CUDA, MR_ERR_TIMEOUT = range(6)
 MR_F16, MR_BF16, MR_F32 = 0, 1, 2
 MR_GEMV_PDL = 0x1
+MR_GEMV_SIGMOID = 0x2
 MR_DEVERR_GEMV_TIMEOUT, MR_DEVERR_GEMM_TIMEOUT, MR_DEVERR_TOPK_TIMEOUT, MR_DEVERR_SELFTEST = 1, 2, 4, 8
 
 EXPORTS = (
     "mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
     "router_gemv_topk_workspace_bytes", "router_gemv_topk_noalloc", "router_gemv_topk_noalloc_max_logits", "gemm_f16_grouped",
-    "gemm_f16_grouped_select_tile", "gemm_f16", "gemm_f16_num_tiles",
+    "gemm_f16_grouped_select_tile", "cast_f32_bf16", "gemm_f16", "gemm_f16_num_tiles",
     "gemm_f16_tile_name", "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout",
     "mr_status_str", "mr_version",
 )
@@ -59,6 +60,7 @@ def _load() -> ctypes.CDLL:
     L.gemm_f16.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, I32, I32, P]
     L.gemm_f16_grouped.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, I32, I32, I32, P]
     L.gemm_f16_grouped_select_tile.argtypes = [I32, I32, I32, I32]
+    L.cast_f32_bf16.argtypes = [P, I64, P, I64, I32, I32, P]
     L.gemm_f16_num_tiles.argtypes = []
     L.gemm_f16_tile_name.argtypes = [I32]
     L.gemm_f16_tile_name.restype = ctypes.c_char_p
@@ -70,7 +72,8 @@ def _load() -> ctypes.CDLL:
     L.mr_version.argtypes = []
     L.mr_version.restype = ctypes.c_char_p
     for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
-                 "router_gemv_topk_noalloc", "gemm_f16_grouped", "gemm_f16_grouped_select_tile", "gemm_f16", "gemm_f16_num_tiles",
+                 "router_gemv_topk_noalloc", "gemm_f16_grouped", "gemm_f16_grouped_select_tile",
+                 "cast_f32_bf16", "gemm_f16", "gemm_f16_num_tiles",
                  "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     return L
@@ -226,6 +229,15 @@ def gemm_f16_grouped(A, Wts, Cs, tile_id: int = -1, in_dtype: int | None = None,
 
 def gemm_f16_grouped_select_tile(M: int, N: int, K: int, G: int) -> int:
     return int(lib.gemm_f16_grouped_select_tile(M, N, K, G))
+
+
+def cast_f32_bf16(X, Y, stream=None) -> None:
+    """Y (bf16 or int16 bits) = X (fp32) rounded to nearest even."""
+    rows, cols, ldx = _rows(X, "X")
+    ry, cy, ldy = _rows(Y, "Y")
+    if (ry, cy) != (rows, cols):
+        raise ValueError("X and Y shapes differ")
+    _check(lib.cast_f32_bf16(X.data_ptr(), ldx, Y.data_ptr(), ldy, rows, cols, _stream(stream)), "cast_f32_bf16")
 
 
 def gemm_f16_num_tiles() -> int:

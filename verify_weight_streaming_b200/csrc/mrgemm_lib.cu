@@ -4,3 +4,4 @@
 #include "mrgemv.cu"
 #include "router_topk.cu"
 #include "gemm_f16.cu"
+#include "cast_bf16.cu"

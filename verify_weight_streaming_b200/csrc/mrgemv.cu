@@ -60,6 +60,7 @@ struct Params {
     int S;          // ring slots
     uint32_t a_bytes;     // shared bytes reserved for A (MB rows)
     uint32_t slot_bytes;  // CG * k * 2
+    int sigmoid;          // store 1 / (1 + exp(-c)) instead of c (MR_GEMV_SIGMOID)
     // Fused router (top-k of each row after the GEMV), unused otherwise.
     int topk;
     int32_t *idx;
@@ -75,6 +76,12 @@ __host__ __device__ inline int k_warps(int k) {
     if (q % 128 == 0 && q >= 512) return 4;
     if (q % 64 == 0 && q >= 256) return 2;
     return 1;
+}
+
+// The shared expert's scalar gate: logistic of the GEMV output, with CUDA's
+// expf and an IEEE divide.
+__device__ __forceinline__ float gate_out(const Params &p, float c) {
+    return p.sigmoid ? 1.0f / (1.0f + expf(-c)) : c;
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -250,7 +257,7 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
             for (int i = 0; i < PL; ++i) {
                 const int idx = base + i;
                 const int r = idx / NC, j = idx % NC;
-                if (r < p.m && j < ncol) p.C[(int64_t)r * p.ldc + col0 + j] = v[i];
+                if (r < p.m && j < ncol) p.C[(int64_t)r * p.ldc + col0 + j] = gate_out(p, v[i]);
             }
         }
     }
@@ -427,7 +434,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p)
                 const float *src = sm.red + (size_t)g * p.KW * VCG + rem;
                 float acc = src[0];
                 for (int sl = 1; sl < p.KW; ++sl) acc = __fadd_rn(acc, src[(size_t)sl * VCG]);
-                p.C[(int64_t)r * p.ldc + col] = acc;
+                p.C[(int64_t)r * p.ldc + col] = gate_out(p, acc);
             }
         }
     }
@@ -619,7 +626,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
 extern "C" mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t flags, int32_t sm_count,
                                       int32_t smem_optin, int32_t *out) {
     if (!out) return MR_ERR_INVALID_ARG;
-    if (flags & ~MR_GEMV_PDL) return MR_ERR_INVALID_ARG;
+    if (flags & ~(MR_GEMV_PDL | MR_GEMV_SIGMOID)) return MR_ERR_INVALID_ARG;
     mr::gemv::Plan pl;
     const mr_status st = mr::gemv::make_plan(m, n, k, flags, sm_count, smem_optin, pl);
     if (st != MR_OK) return st;
@@ -651,7 +658,8 @@ mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float 
     if (!A || !Wt || !C) return MR_ERR_INVALID_ARG;
     if (m < 1 || n < 1 || k < 1) return MR_ERR_INVALID_ARG;
     if (lda < k || ldw < k || ldc < n) return MR_ERR_INVALID_ARG;
-    if (flags & ~MR_GEMV_PDL) return MR_ERR_INVALID_ARG;
+    if (flags & ~(MR_GEMV_PDL | MR_GEMV_SIGMOID)) return MR_ERR_INVALID_ARG;
+    if (fused && (flags & MR_GEMV_SIGMOID)) return MR_ERR_INVALID_ARG;
     if (k % 8 != 0 || lda % 8 != 0 || ldw % 8 != 0) return MR_ERR_MISALIGNED;
     if (((uintptr_t)A & 15u) || ((uintptr_t)Wt & 15u) || ((uintptr_t)C & 3u)) return MR_ERR_MISALIGNED;
     if (m > kMaxRows) return MR_ERR_UNSUPPORTED;
@@ -682,6 +690,7 @@ mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float 
     p.S = pl.S;
     p.a_bytes = pl.a_bytes;
     p.slot_bytes = pl.slot_bytes;
+    p.sigmoid = (flags & MR_GEMV_SIGMOID) ? 1 : 0;
     if (fused) {
         p.topk = fused->topk;
         p.idx = fused->idx;
