@@ -655,6 +655,23 @@ def gemm_sweep(quick=False):
                                  "grouped_TFLOPs": 36 * 2.0 * M * 96 * K / (ug * 1e-6) / 1e12,
                                  "grouped_tile": mr.gemm_f16_tile_name(
                                      mr.gemm_f16_grouped_select_tile(M, 96, K, 36))}
+    # Tile-order study (the analogue of the audit's SLC swizzle): same bits,
+    # timed for several column-band widths.
+    study = {}
+    for (M, N) in ((2048, 6144), (1983, 4096), (448, 6144)):
+        A = a_all[:M]
+        W = w_all[:N]
+        ref = None
+        row = {}
+        for raster in (0, 2, 4, 8):
+            C = torch.empty((M, N), dtype=torch.float16, device="cuda")
+            us = _time_calls(torch, [lambda C=C, r=raster: mr.gemm_f16(A, W, C, raster=r)] * 8)
+            torch.cuda.synchronize()
+            same = True if ref is None else bool(torch.equal(C.view(torch.int16), ref.view(torch.int16)))
+            ref = C if ref is None else ref
+            row[str(raster)] = {"us": us, "TFLOPs": 2.0 * M * N * K / (us * 1e-6) / 1e12, "same_bits": same}
+        study[f"{M}x{N}"] = row
+    out["raster_study"] = study
     out["summary"] = {"tflops_M_ge_1024_mean": float(np.mean(big)) if big else None,
                       "tflops_M_ge_1024_max": float(np.max(big)) if big else None,
                       "peak_bf16_tflops": tf_burst, "peak_kind": kind,

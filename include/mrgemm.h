@@ -228,6 +228,19 @@ mr_status gemm_f16(const void *A, int64_t lda, const void *Wt, int64_t ldw,
                    void *stream);
 
 /*
+ * gemm_f16_ex -- gemm_f16 with a tile order: raster 0 is the default (a row
+ * tile's N tiles, then the next row tile); raster R in 1..64 walks bands of R
+ * N tiles down every row tile, the column-band order of the audit's SLC
+ * swizzle study ("opus r35 track A", section 2, SLC swizzle).  Outputs are
+ * bitwise identical for every raster; only the order of tiles, and so the
+ * reuse of operands in L2, changes.
+ */
+mr_status gemm_f16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw,
+                      void *C, int64_t ldc, int32_t M, int32_t N, int32_t K,
+                      int32_t in_dtype, int32_t out_dtype, int32_t tile_id, int32_t raster,
+                      void *stream);
+
+/*
  * gemm_f16_grouped -- G GEMMs that share A in one launch: for g < G,
  *   Cs[g][i][j] = sum_p A[i][p] * Wts[g][j][p]
  * The 36 independent N = 96 projections of one prompt chunk in the

@@ -167,3 +167,10 @@ def test_gate_flag_validation():
     st = mr.lib.router_gemv_topk(A16, 64, A16, 64, None, 512, 4, 512, 64, 10, A16, None, 10, P(512),
                                  1 << 20, mr.MR_GEMV_SIGMOID, None)
     assert st == mr.MR_ERR_INVALID_ARG
+
+
+def test_gemm_raster_validation():
+    g = mr.lib.gemm_f16_ex
+    assert g(A16, 64, A16, 64, A16, 32, 4, 32, 64, 0, 0, -1, -1, None) == mr.MR_ERR_INVALID_ARG
+    assert g(A16, 64, A16, 64, A16, 32, 4, 32, 64, 0, 0, -1, 65, None) == mr.MR_ERR_INVALID_ARG
+    assert g(A16, 64, A16, 64, A16, 32, 4, 32, 64, 0, 0, -1, 8, None) == mr.MR_ERR_CUDA  # valid; no device

@@ -196,3 +196,21 @@ def test_grouped_every_tile_bitwise(G, N, K):
         outs = run_grouped(a, ws, fmt="bf16", out_fmt="bf16", tile=tile)
         for g in range(G):
             assert np.array_equal(outs[g], refs[g]), (tile, g)
+
+
+@pytest.mark.parametrize("M,N,tile", [(700, 640, 0), (1983, 1152, 3), (300, 2000, 5), (129, 96, 2)])
+def test_raster_orders_give_identical_bits(M, N, tile):
+    """Tile order (the SLC-swizzle analogue) changes only the schedule."""
+    a = synth.normal_bits(41, (M, 2560), "f16", 1.0)
+    w = synth.normal_bits(42, (N, 2560), "f16", 1.0 / np.sqrt(2560))
+    A, W = dev_bits(a, torch.float16), dev_bits(w, torch.float16)
+    ldc = (N + 7) // 8 * 8
+    ref = None
+    for raster in (0, 1, 2, 3, 8, 64):
+        C = torch.full((M, ldc), float("nan"), dtype=torch.float16, device="cuda")
+        mr.gemm_f16(A, W, C[:, :N], tile_id=tile, raster=raster)
+        raw = host(C.view(torch.int16))[:, :N]
+        if ref is None:
+            ref = raw
+            check(synth.bits_to_float32(raw.view(np.uint16), "f16")[:64], a[:64], w, "f16", "f16")
+        assert np.array_equal(raw, ref), raster

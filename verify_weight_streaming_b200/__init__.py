@@ -23,7 +23,7 @@ MR_DEVERR_GEMV_TIMEOUT, MR_DEVERR_GEMM_TIMEOUT, MR_DEVERR_TOPK_TIMEOUT, MR_DEVER
 EXPORTS = (
     "mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
     "router_gemv_topk_workspace_bytes", "router_gemv_topk_noalloc", "router_gemv_topk_noalloc_max_logits", "gemm_f16_grouped",
-    "gemm_f16_grouped_select_tile", "cast_f32_bf16", "gemm_f16", "gemm_f16_num_tiles",
+    "gemm_f16_grouped_select_tile", "cast_f32_bf16", "gemm_f16_ex", "gemm_f16", "gemm_f16_num_tiles",
     "gemm_f16_tile_name", "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout",
     "mr_status_str", "mr_version",
 )
@@ -61,6 +61,7 @@ def _load() -> ctypes.CDLL:
     L.gemm_f16_grouped.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, I32, I32, I32, P]
     L.gemm_f16_grouped_select_tile.argtypes = [I32, I32, I32, I32]
     L.cast_f32_bf16.argtypes = [P, I64, P, I64, I32, I32, P]
+    L.gemm_f16_ex.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, I32, I32, I32, P]
     L.gemm_f16_num_tiles.argtypes = []
     L.gemm_f16_tile_name.argtypes = [I32]
     L.gemm_f16_tile_name.restype = ctypes.c_char_p
@@ -73,7 +74,7 @@ def _load() -> ctypes.CDLL:
     L.mr_version.restype = ctypes.c_char_p
     for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
                  "router_gemv_topk_noalloc", "gemm_f16_grouped", "gemm_f16_grouped_select_tile",
-                 "cast_f32_bf16", "gemm_f16", "gemm_f16_num_tiles",
+                 "cast_f32_bf16", "gemm_f16_ex", "gemm_f16", "gemm_f16_num_tiles",
                  "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     return L
@@ -195,7 +196,7 @@ def router_gemv_topk(A, Wt, topk: int, idx, val=None, logits=None, workspace=Non
     _check(st, "router_gemv_topk")
 
 
-def gemm_f16(A, Wt, C, tile_id: int = -1, in_dtype: int | None = None, stream=None) -> None:
+def gemm_f16(A, Wt, C, tile_id: int = -1, in_dtype: int | None = None, stream=None, raster: int = 0) -> None:
     """C[M,N] = A[M,K] . Wt[N,K]^T on tcgen05; dtypes from the tensors (int16 = bf16 bits)."""
     M, K, lda = _rows(A, "A")
     N, kw, ldw = _rows(Wt, "Wt")
@@ -203,8 +204,8 @@ def gemm_f16(A, Wt, C, tile_id: int = -1, in_dtype: int | None = None, stream=No
     if kw != K or mc != M or nc != N:
         raise ValueError("shape mismatch")
     idt = _dtype_code(A) if in_dtype is None else in_dtype
-    st = lib.gemm_f16(A.data_ptr(), lda, Wt.data_ptr(), ldw, C.data_ptr(), ldc, M, N, K,
-                      idt, _dtype_code(C), tile_id, _stream(stream))
+    st = lib.gemm_f16_ex(A.data_ptr(), lda, Wt.data_ptr(), ldw, C.data_ptr(), ldc, M, N, K,
+                         idt, _dtype_code(C), tile_id, raster, _stream(stream))
     _check(st, "gemm_f16")
 
 

@@ -184,8 +184,27 @@ struct GemmArgs {
     int64_t ldc;
     int M, N, K;
     int G, P, tn_per_group, ntn;
+    int raster;     // 0: N-slots fastest; R > 0: bands of R N-slots run down all row tiles
     uint32_t idesc;
 };
+
+// Tile t of the persistent walk -> (row tile, N-slot).  raster == 0 walks the
+// N-slots of a row tile before the next row tile; raster R > 0 walks bands of
+// R N-slots down every row tile (the column-band order of the audit's SLC
+// swizzle study).  Only the order changes, never a tile's arithmetic.
+__device__ __forceinline__ void tile_coords(int t, int ntm, int ntn, int raster, int &mt, int &nt) {
+    if (raster <= 0) {
+        mt = t / ntn;
+        nt = t % ntn;
+        return;
+    }
+    const int band = t / (ntm * raster);
+    const int n0 = band * raster;
+    const int width = min(raster, ntn - n0);
+    const int r = t - band * ntm * raster;
+    mt = r / width;
+    nt = n0 + r % width;
+}
 
 template <int BN, int STAGES, int ACC_COLS, int OUT, int MAXG>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs<MAXG> args) {
@@ -214,7 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int ntn = args.ntn;
-    const int ntiles = ((M + BM - 1) / BM) * ntn;
+    const int ntm = (M + BM - 1) / BM;
+    const int ntiles = ntm * ntn;
     const int nkb = (K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
@@ -245,7 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         uint32_t it = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const int m0 = (t / ntn) * BM, slot = t % ntn;
+            int mt, slot;
+            tile_coords(t, ntm, ntn, args.raster, mt, slot);
+            const int m0 = mt * BM;
             // Groups of this tile and the B rows each contributes.
             const int g0 = P > 1 ? slot * P : slot / args.tn_per_group;
             const int ng = P > 1 ? min(P, G - g0) : 1;
@@ -304,7 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         uint32_t ti = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++ti) {
             const uint32_t b = ti & 1u;
-            const int m0 = (t / ntn) * BM, slot = t % ntn;
+            int mt, slot;
+            tile_coords(t, ntm, ntn, args.raster, mt, slot);
+            const int m0 = mt * BM;
             const int g0 = P > 1 ? slot * P : slot / args.tn_per_group;
             const int n0 = P > 1 ? 0 : (slot % args.tn_per_group) * BN;
             const int row = m0 + 32 * q + lane;
@@ -472,13 +496,14 @@ int select_tile(int M, int N, int K, int sms) { return select_tile_grouped(M, N,
 template <int MAXG>
 mr_status launch(const void *A, int64_t lda, const void *const *Wts, int64_t ldw, void *const *Cs, int64_t ldc,
                  int32_t M, int32_t N, int32_t K, int32_t G, int32_t in_dtype, int32_t out_dtype, int32_t tile_id,
-                 void *stream) {
+                 int32_t raster, void *stream) {
     if (!A || !Wts || !Cs) return MR_ERR_INVALID_ARG;
     if (M < 1 || N < 1 || K < 1 || G < 1 || G > MAXG) return MR_ERR_INVALID_ARG;
     if (lda < K || ldw < K || ldc < N) return MR_ERR_INVALID_ARG;
     if (in_dtype != MR_F16 && in_dtype != MR_BF16) return MR_ERR_INVALID_ARG;
     if (out_dtype != MR_F16 && out_dtype != MR_BF16 && out_dtype != MR_F32) return MR_ERR_INVALID_ARG;
     if (tile_id < -1 || tile_id >= kNumTiles) return MR_ERR_INVALID_ARG;
+    if (raster < 0 || raster > 64) return MR_ERR_INVALID_ARG;
     for (int g = 0; g < G; ++g)
         if (!Wts[g] || !Cs[g]) return MR_ERR_INVALID_ARG;
     if (K % 8 != 0 || lda % 8 != 0 || ldw % 8 != 0 || ldc % 8 != 0) return MR_ERR_MISALIGNED;
@@ -506,6 +531,7 @@ mr_status launch(const void *A, int64_t lda, const void *const *Wts, int64_t ldw
     args.K = K;
     args.G = G;
     args.ldc = ldc;
+    args.raster = raster;
     args.idesc = make_idesc(in_dtype, td.bn);
     if (!encode_operand(&args.tmA, A, M, K, lda, in_dtype, BM)) return MR_ERR_CUDA;
     const int b_rows = args.P > 1 ? N : td.bn;
@@ -540,13 +566,19 @@ extern "C" int32_t gemm_f16_select_tile(int32_t M, int32_t N, int32_t K) {
     return mr::gemm::select_tile(M, N, K, sms);
 }
 
-extern "C" mr_status gemm_f16(const void *A, int64_t lda, const void *Wt, int64_t ldw, void *C, int64_t ldc,
-                              int32_t M, int32_t N, int32_t K, int32_t in_dtype, int32_t out_dtype, int32_t tile_id,
-                              void *stream) {
+extern "C" mr_status gemm_f16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw, void *C, int64_t ldc,
+                                 int32_t M, int32_t N, int32_t K, int32_t in_dtype, int32_t out_dtype, int32_t tile_id,
+                                 int32_t raster, void *stream) {
     const void *w[1] = {Wt};
     void *c[1] = {C};
     if (!Wt || !C) return MR_ERR_INVALID_ARG;
-    return mr::gemm::launch<1>(A, lda, w, ldw, c, ldc, M, N, K, 1, in_dtype, out_dtype, tile_id, stream);
+    return mr::gemm::launch<1>(A, lda, w, ldw, c, ldc, M, N, K, 1, in_dtype, out_dtype, tile_id, raster, stream);
+}
+
+extern "C" mr_status gemm_f16(const void *A, int64_t lda, const void *Wt, int64_t ldw, void *C, int64_t ldc,
+                              int32_t M, int32_t N, int32_t K, int32_t in_dtype, int32_t out_dtype, int32_t tile_id,
+                              void *stream) {
+    return gemm_f16_ex(A, lda, Wt, ldw, C, ldc, M, N, K, in_dtype, out_dtype, tile_id, 0, stream);
 }
 
 extern "C" mr_status gemm_f16_grouped(const void *A, int64_t lda, const void *const *Wts, int64_t ldw, void *const *Cs,
@@ -554,7 +586,7 @@ extern "C" mr_status gemm_f16_grouped(const void *A, int64_t lda, const void *co
                                       int32_t out_dtype, int32_t tile_id, void *stream) {
     if (G > mr::gemm::kMaxGroups) return MR_ERR_UNSUPPORTED;
     return mr::gemm::launch<mr::gemm::kMaxGroups>(A, lda, Wts, ldw, Cs, ldc, M, N, K, G, in_dtype, out_dtype,
-                                                  tile_id, stream);
+                                                  tile_id, 0, stream);
 }
 
 extern "C" int32_t gemm_f16_grouped_select_tile(int32_t M, int32_t N, int32_t K, int32_t G) {
