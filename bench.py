@@ -393,8 +393,9 @@ def run_gpu(args, world, rank, local):
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(rb, args, world, device, fused=(best_form == "fused"))
 
-    # ---- GEMM sweep (prompt-chunk shapes)
+    # ---- GEMM sweep (prompt-chunk shapes) and the m-sweep over both paths
     gemm = run_gemm_sweep(args) if not args.skip_gemm else None
+    sweep = path_sweep() if not (args.skip_gemm or args.quick) else None
 
     # ---- CPU oracle baseline (rank 0, N=1 only)
     cpu = None
@@ -412,7 +413,7 @@ def run_gpu(args, world, rank, local):
             "forms_us_per_row": forms_us_per_row,
             "device_errors": errs, "clocks": clocks_best, "roofline": roofline,
             "curve": {"router": curve, "batching_speedup_m1_over_m8": speedup, **extra_curves},
-            "e2e": e2e, "gemm": gemm, "cpu_baseline": cpu,
+            "e2e": e2e, "gemm": gemm, "path_sweep": sweep, "cpu_baseline": cpu,
             "pdl": not args.no_pdl,
         }
         print(json.dumps(line), flush=True)
@@ -677,6 +678,59 @@ def gemm_sweep(quick=False):
                       "peak_bf16_tflops": tf_burst, "peak_kind": kind,
                       "frac_of_peak_mean": (float(np.mean(big)) / tf_burst) if big else None}
     return out
+
+
+SWEEP_M = (1, 2, 4, 8, 16, 32, 64, 128, 256, 306, 512, 1024, 1983, 2048)
+
+
+def path_sweep():
+    """The m-sweep over both paths on the FFN (k=896, n=4864) and the
+    (k=2560, n=6144) weights: us_per_row of the multi-row GEMV (m > 16 runs as
+    16-row groups, each re-reading the weight) and of the tcgen05 GEMM (bf16
+    in, fp32 out, auto tile), and the smallest m at which the GEMM is faster.
+    Weights rotate over copies larger than 2x L2."""
+    import numpy as np
+    import torch
+    import synth
+    import verify_weight_streaming_b200 as mr
+    props = torch.cuda.get_device_properties(0)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    res = {}
+    for name, k, n, wl in (("k896_n4864", 896, 4864, synth.WL_GEMV_FFN),
+                           ("k2560_n6144", 2560, 6144, synth.WL_SWEEP)):
+        a16 = synth.normal_bits(synth.seed_for(wl, 0), (max(SWEEP_M), k), "bf16", 1.0)
+        w16 = synth.normal_bits(synth.seed_for(wl, 1), (n, k), "bf16", 1.0 / np.sqrt(k))
+        A = torch.from_numpy(a16.view(np.int16)).cuda()
+        w = torch.from_numpy(w16.view(np.int16)).cuda()
+        copies = max(3, int(np.ceil(2.2 * l2 / w16.nbytes)))
+        Ws = [w.clone() for _ in range(copies)]
+        Ab = A.view(torch.bfloat16)
+        Wb = [x.view(torch.bfloat16) for x in Ws]
+        curve = {}
+        cross = None
+        for m in SWEEP_M:
+            C = torch.empty((m, n), dtype=torch.float32, device="cuda")
+            groups = [(r0, min(16, m - r0)) for r0 in range(0, m, 16)]
+            calls = []
+            for i in range(copies):
+                def gemv_call(i=i):
+                    for r0, rr in groups:
+                        mr.mrgemv_bf16(A[r0:r0 + rr], Ws[i], C[r0:r0 + rr], flags=mr.MR_GEMV_PDL)
+                calls.append(gemv_call)
+            t_gemv = _time_calls(torch, calls, reps=2)
+            gcalls = [(lambda i=i: mr.gemm_f16(Ab[:m], Wb[i], C)) for i in range(copies)]
+            t_gemm = _time_calls(torch, gcalls, reps=2)
+            curve[str(m)] = {"gemv_us_per_row": t_gemv / m, "gemm_us_per_row": t_gemm / m,
+                             "gemv_us": t_gemv, "gemm_us": t_gemm,
+                             "gemm_TFLOPs": 2.0 * m * n * k / (t_gemm * 1e-6) / 1e12,
+                             "gemm_tile": mr.gemm_f16_tile_name(mr.gemm_f16_select_tile(m, n, k))}
+            if cross is None and t_gemm <= t_gemv:
+                cross = m
+            del C
+        res[name] = {"curve": curve, "crossover_m": cross,
+                     "note": "GEMV for m > 16 is ceil(m/16) calls of up to 16 rows; GEMM is one call"}
+        del Ws, Wb, w
+    return res
 
 
 def gemm_profile_case():
