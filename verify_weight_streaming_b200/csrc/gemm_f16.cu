@@ -5,14 +5,17 @@
 // tiles (M % 128 in 1..64), and outputs that are bitwise identical whatever
 // tile is chosen.  Rebuilt for B200:
 //
-//  * persistent CTAs (one per SM) walk the 128 x BN output tiles; 6 warps:
-//    warp 0 issues TMA loads, warp 1 owns the tensor memory and issues
-//    tcgen05.mma from one thread, warps 2..5 drain the accumulator
+//  * persistent CTAs (one per SM) walk the 128 x BN output tiles; 7 warps:
+//    warps 0 and 6 issue TMA loads, warp 1 owns the tensor memory and issues
+//    tcgen05.mma from one elected thread, warps 2..5 drain the accumulator
 //    (tcgen05.ld) and store the tile.  Two accumulator buffers in tensor
 //    memory let one tile's epilogue run under the next tile's MMAs;
-//  * A and Wt tiles of 64 K-elements (one 128-byte swizzle atom per row) are
-//    loaded by TMA (no multicast) into a ring of STAGES shared-memory stages,
-//    full/empty mbarriers between the producer and the MMA thread;
+//  * A and Wt k-blocks of 64 K-elements (one 128-byte swizzle atom per row)
+//    are loaded by TMA (no multicast) into a ring of shared-memory stages,
+//    full/empty mbarriers between the producers and the MMA thread.  Each
+//    ring step (barrier wait, TMA or MMA issue, commit) costs a few hundred
+//    cycles of latency: two producer warps alternate stages, and the narrow
+//    tiles, whose MMAs are short, put two k-blocks in a stage;
 //  * tcgen05.mma.cta_group::1.kind::f16 with M = 128, N = BN, K = 16,
 //    accumulating fp32 in tensor memory.  Every tile runs the same sequence of
 //    K steps (16 at a time, ascending, zero padding past K), with no split-K
@@ -37,20 +40,28 @@ namespace mr {
 namespace gemm {
 
 constexpr int BM = 128;          // rows per tile (MMA M)
-constexpr int BK = 64;           // K elements per stage (128 bytes of 16-bit data)
-constexpr int kThreads = 192;    // 6 warps
+constexpr int BK = 64;           // K elements per k-block (128 bytes of 16-bit data)
 constexpr uint32_t kABytes = BM * BK * 2;
+
+// Threads of a CTA: warps 0 and 6 producers (alternate ring stages), warp 1
+// MMA issue, warps 2-5 epilogue.
+constexpr int kThreads = 224;
+constexpr int kProducers = 2;
 
 struct TileDesc {
     int bn;
-    int stages;
+    int stages;     // k-block slots of shared memory
     int acc_cols;   // tensor-memory columns per accumulator buffer (power of two >= bn)
+    int kpb;        // k-blocks per ring stage (one barrier wait and one commit each)
     const char *name;
 };
 
+// Narrow tiles take two k-blocks per ring stage: their MMAs are short (the
+// operand reads from shared memory bound them), so one barrier round trip and
+// one commit per k-block would leave the tensor pipe idle between stages.
 constexpr TileDesc kTiles[] = {
-    {32, 8, 32, "128x32"},   {64, 8, 64, "128x64"},   {96, 7, 128, "128x96"},
-    {128, 6, 128, "128x128"}, {192, 5, 256, "128x192"}, {256, 4, 256, "128x256"},
+    {32, 8, 32, 2, "128x32"},   {64, 8, 64, 2, "128x64"},   {96, 7, 128, 1, "128x96"},
+    {128, 6, 128, 1, "128x128"}, {192, 5, 256, 1, "128x192"}, {256, 4, 256, 1, "128x256"},
 };
 constexpr int kNumTiles = sizeof(kTiles) / sizeof(kTiles[0]);
 
@@ -90,6 +101,18 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     d |= (uint64_t)1u << 46;
     d |= (uint64_t)2u << 61;
     return d;
+}
+
+// One lane of a converged warp (the one elect.sync picks); the MMA issue
+// branch is taken by exactly one thread.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
 }
 
 __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -206,7 +229,7 @@ __device__ __forceinline__ void tile_coords(int t, int ntm, int ntn, int raster,
     nt = n0 + r % width;
 }
 
-template <int BN, int STAGES, int ACC_COLS, int OUT, int MAXG>
+template <int BN, int STAGES, int ACC_COLS, int KPB, int OUT, int MAXG>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs<MAXG> args) {
     const CUtensorMap &tmA = args.tmA;
     const int M = args.M, N = args.N, K = args.K, G = args.G, P = args.P;
@@ -224,8 +247,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     const uint32_t sA = base;
     const uint32_t sB = base + STAGES * kABytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + STAGES * (kABytes + kBBytes));
-    uint64_t *full = bars;                    // [STAGES] TMA -> MMA
-    uint64_t *empty = bars + STAGES;          // [STAGES] MMA -> TMA
+    // Ring of NST stages of KPB k-blocks each (k-block slot j of stage s is
+    // slot s * KPB + j of the A and B regions).  Producer p issues the stages
+    // it with it % kProducers == p.  Its previous stage was it - kProducers,
+    // whose wait saw stage it - kProducers - NST released; with NST >=
+    // kProducers that covers stage it - 2 NST, so a wait on a slot is never
+    // more than one phase ahead of the barrier.
+    constexpr int NST = STAGES / KPB;
+    static_assert(NST >= kProducers, "ring too short for the producer warps");
+    uint64_t *full = bars;                    // [NST] TMA -> MMA
+    uint64_t *empty = bars + STAGES;          // [NST] MMA -> TMA
     uint64_t *acc_full = bars + 2 * STAGES;   // [2] MMA -> epilogue
     uint64_t *acc_empty = bars + 2 * STAGES + 2;  // [2] epilogue -> MMA
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
@@ -236,9 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     const int ntm = (M + BM - 1) / BM;
     const int ntiles = ntm * ntn;
     const int nkb = (K + BK - 1) / BK;
+    const int nst = (nkb + KPB - 1) / KPB;   // ring stages per tile
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
             mbar_init(smem_u32(&empty[s]), 1);
         }
@@ -259,9 +291,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     // Warps 0 and 1 run their loops as whole warps (every lane waits on the
     // same barrier) and let lane 0 issue: a lone lane spinning in try_wait
     // beside warp-mates parked elsewhere can stall for the suspend limit.
-    if (warp == 0) {
-        // Producer: k-block `it` counts across tiles, so stages and phases
+    if (warp == 0 || warp == 6) {
+        // Producers: stage `it` counts across tiles, so slots and phases
         // continue from one tile to the next.
+        const uint32_t pidx = warp == 0 ? 0u : 1u;
         uint32_t it = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
@@ -273,24 +306,35 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const int ng = P > 1 ? min(P, G - g0) : 1;
             const int n0 = P > 1 ? 0 : (slot % args.tn_per_group) * BN;
             const uint32_t b_rows = P > 1 ? (uint32_t)N : (uint32_t)BN;
-            const uint32_t tx = kABytes + (uint32_t)ng * b_rows * BK * 2;
-            for (int kb = 0; kb < nkb; ++kb, ++it) {
-                const uint32_t s = it % STAGES;
-                const uint32_t par = ((it / STAGES) & 1u) ^ 1u;
+            const uint32_t kb_bytes = kABytes + (uint32_t)ng * b_rows * BK * 2;
+            for (int ks = 0; ks < nst; ++ks, ++it) {
+                if (it % kProducers != pidx) continue;
+                const uint32_t s = it % NST;
+                const uint32_t par = ((it / NST) & 1u) ^ 1u;
+                const int nsub = KPB == 1 ? 1 : min(KPB, nkb - ks * KPB);
                 ok = mbar_wait_bounded(smem_u32(&empty[s]), par, MR_DEVERR_GEMM_TIMEOUT);
                 if (!ok) break;
                 if (lane == 0) {
                     const uint32_t fb = smem_u32(&full[s]);
-                    mbar_arrive_expect_tx(fb, tx);
-                    tma_load_2d(sA + s * kABytes, &tmA, kb * BK, m0, fb);
-                    for (int j = 0; j < ng; ++j)
-                        tma_load_2d(sB + s * kBBytes + (uint32_t)j * b_rows * BK * 2, &args.tmB[g0 + j], kb * BK,
-                                    n0, fb);
+                    mbar_arrive_expect_tx(fb, (uint32_t)nsub * kb_bytes);
+#pragma unroll
+                    for (int sub = 0; sub < KPB; ++sub) {
+                        if (sub >= nsub) break;
+                        const int kb = ks * KPB + sub;
+                        const uint32_t slot_kb = s * KPB + (uint32_t)sub;
+                        tma_load_2d(sA + slot_kb * kABytes, &tmA, kb * BK, m0, fb);
+                        for (int j = 0; j < ng; ++j)
+                            tma_load_2d(sB + slot_kb * kBBytes + (uint32_t)j * b_rows * BK * 2, &args.tmB[g0 + j],
+                                        kb * BK, n0, fb);
+                    }
                 }
                 __syncwarp();
             }
         }
     } else if (warp == 1) {
+        // Descriptors of slot 0; a slot's descriptor adds its byte offset >> 4
+        // to the start-address field (shared addresses stay below 2^18).
+        const uint64_t adesc0 = sw128_desc(sA), bdesc0 = sw128_desc(sB);
         uint32_t it = 0, ti = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++ti) {
@@ -300,18 +344,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             if (!ok) break;
             tc_fence_after();
             const uint32_t acc = tmem + b * ACC_COLS;
-            for (int kb = 0; kb < nkb; ++kb, ++it) {
-                const uint32_t s = it % STAGES;
-                const uint32_t par = (it / STAGES) & 1u;
+            for (int ks = 0; ks < nst; ++ks, ++it) {
+                const uint32_t s = it % NST;
+                const uint32_t par = (it / NST) & 1u;
+                const int nsub = KPB == 1 ? 1 : min(KPB, nkb - ks * KPB);
                 ok = mbar_wait_bounded(smem_u32(&full[s]), par, MR_DEVERR_GEMM_TIMEOUT);
                 if (!ok) break;
                 tc_fence_after();
-                if (lane == 0) {
+                __syncwarp();
+                if (elect_one()) {
+                    // K steps of 16 in ascending order: every tile and every
+                    // stage grouping issues the same MMA sequence.
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t ad = sw128_desc(sA + s * kABytes + kk * 32);
-                        const uint64_t bd = sw128_desc(sB + s * kBBytes + kk * 32);
-                        mma_f16(acc, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    for (int sub = 0; sub < KPB; ++sub) {
+                        if (sub >= nsub) break;
+                        const uint32_t slot_kb = s * KPB + (uint32_t)sub;
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t ad = adesc0 + (uint64_t)((slot_kb * kABytes + kk * 32) >> 4);
+                            const uint64_t bd = bdesc0 + (uint64_t)((slot_kb * kBBytes + kk * 32) >> 4);
+                            mma_f16(acc, ad, bd, idesc, (ks | sub | kk) != 0 ? 1u : 0u);
+                        }
                     }
                     mma_commit(smem_u32(&empty[s]));
                 }
@@ -368,7 +421,7 @@ using KernelFn = void (*)(const GemmArgs<MAXG>);
 
 template <int T, int OUT, int MAXG>
 constexpr KernelFn<MAXG> kernel_of() {
-    return gemm_kernel<kTiles[T].bn, kTiles[T].stages, kTiles[T].acc_cols, OUT, MAXG>;
+    return gemm_kernel<kTiles[T].bn, kTiles[T].stages, kTiles[T].acc_cols, kTiles[T].kpb, OUT, MAXG>;
 }
 
 template <int OUT, int MAXG>
