@@ -16,6 +16,7 @@ and the SM clocks seen during the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
     python bench.py --profile-case gemv|topk|gemm   # a few launches, for ncu
+    python bench.py --selector-study                # every GEMM tile on every chunk shape
 """
 from __future__ import annotations
 
@@ -680,6 +681,44 @@ def gemm_sweep(quick=False):
     return out
 
 
+def selector_study():
+    """Every tile of gemm_f16 timed on every prompt-chunk shape, against the
+    tile the selector picks: regret = t(selected) / t(best) - 1.  Timed like
+    gemm_sweep (graph replays over operand copies larger than twice the L2).
+    All tiles give the same bits, so this only measures the selection rule."""
+    import numpy as np
+    import torch
+    import synth
+    import verify_weight_streaming_b200 as mr
+    props = torch.cuda.get_device_properties(0)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    K = 2560
+    a_all = torch.from_numpy(synth.chunk(max(GEMM_M), 16)[0].view(np.int16)).cuda().view(torch.float16)
+    w_all = torch.from_numpy(synth.chunk(16, max(GEMM_N))[1].view(np.int16)).cuda().view(torch.float16)
+    names = [mr.gemm_f16_tile_name(t) for t in range(mr.gemm_f16_num_tiles())]
+    shapes, regrets = {}, []
+    for N in GEMM_N:
+        for M in GEMM_M:
+            per = (M + N) * K * 2
+            copies = int(min(48, max(2, np.ceil(2.2 * l2 / per))))
+            As = [a_all[:M].clone() for _ in range(copies)]
+            Ws = [w_all[:N].clone() for _ in range(copies)]
+            C = torch.empty((M, N), dtype=torch.float16, device="cuda")
+            times = {}
+            for t, name in enumerate(names):
+                calls = [(lambda A=As[i], W=Ws[i], t=t: mr.gemm_f16(A, W, C, tile_id=t)) for i in range(copies)]
+                times[name] = _time_calls(torch, calls)
+            sel = names[mr.gemm_f16_select_tile(M, N, K)]
+            best = min(times, key=times.get)
+            regret = times[sel] / times[best] - 1.0
+            regrets.append(regret)
+            shapes[f"{M}x{N}"] = {"us": times, "selected": sel, "best": best, "regret": regret}
+            del As, Ws, C
+    return {"K": K, "shapes": shapes,
+            "summary": {"mean_regret": float(np.mean(regrets)), "max_regret": float(np.max(regrets)),
+                        "best_picked": int(sum(1 for r in regrets if r <= 1e-9)), "shapes": len(regrets)}}
+
+
 SWEEP_M = (1, 2, 4, 8, 16, 32, 64, 128, 256, 306, 512, 1024, 1983, 2048)
 
 
@@ -818,12 +857,16 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--quick", action="store_true")
     ap.add_argument("--profile-case", default=None)
+    ap.add_argument("--selector-study", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_env()
     if args.profile_case:
         profile_case(args.profile_case)
+        return
+    if args.selector_study:
+        print(json.dumps(selector_study()), flush=True)
         return
     if args.impl == "reference":
         line = run_reference(args, world, rank)

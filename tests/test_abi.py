@@ -111,6 +111,25 @@ def test_gemm_tiles_and_selector_on_host():
             assert 0 <= mr.gemm_f16_select_tile(M, N, 2560) < n
 
 
+def test_selector_tail_rule_and_measured_choices():
+    """Row tails count as whole 128-row tiles: every M with the same number of
+    row tiles gets the same tile.  And on shapes where one tile was clearly
+    fastest in the all-tiles timing on a B200 (bench.py --selector-study,
+    K = 2560, operands from HBM; the runner-up at least 8% slower), the
+    selector picks it."""
+    names = [mr.gemm_f16_tile_name(t) for t in range(mr.gemm_f16_num_tiles())]
+    for N in (512, 1152, 4096, 6144):
+        for rt in (2, 5, 11, 16):
+            picks = {mr.gemm_f16_select_tile(M, N, 2560) for M in (128 * (rt - 1) + 1, 128 * rt - 64, 128 * rt)}
+            assert len(picks) == 1, (N, rt, picks)
+    measured_best = {(150, 512): "128x32", (1300, 512): "128x64", (1983, 1664): "128x192",
+                     (1300, 4096): "128x192", (306, 6144): "128x128", (2048, 4096): "128x256",
+                     (700, 6144): "128x256", (448, 4096): "128x128", (150, 4096): "128x64",
+                     (1983, 1152): "128x128", (448, 6144): "128x192"}
+    for (M, N), name in measured_best.items():
+        assert names[mr.gemm_f16_select_tile(M, N, 2560)] == name, (M, N)
+
+
 def fused(A=A16, W=A16, logits=None, m=4, n=512, k=64, topk=10, idx=A16, ldo=10, ws=P(512), wsb=1 << 20):
     return mr.lib.router_gemv_topk(A, 64, W, 64, logits, 512, m, n, k, topk, idx, None, ldo, ws, wsb, 0, None)
 

@@ -495,16 +495,16 @@ uint32_t make_idesc(int in_dtype, int bn) {
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
-// Tile selection: estimated time = waves x per-tile time, a wave being one
-// tile on every active SM.  Per-tile time is the larger of
-//  * the padded MMA work of the tile at a rate that grows with BN (wider tiles
-//    reuse each A stage for more columns) plus a small fixed cost, and
-//  * streaming the tile's operands into the SM, (128 + BN) x K x 2 bytes, at
-//    the per-SM share of the measured copy bandwidth (at most ~100 GB/s per SM).
-// Row tails count as whole 128-row tiles, so an M with a small M % 128 pays for
-// the padding it creates (the audit's tail-tile rule); narrow N (the N = 96
-// projections) is bounded by the operand stream and favours spreading tiles
-// over more SMs.
+// Tile selection: estimated time = waves x k-blocks x the tile's time per
+// k-block, a wave being one tile on every active SM.  The per-k-block times
+// are measured: every tile timed on the 48 prompt-chunk shapes (M = 150..2048,
+// N = 512..6144, K = 2560, operands from HBM) runs at a near-constant cost per
+// wave, and these are those costs / 40 k-blocks.  Narrow tiles are cheap per
+// wave (two k-blocks per ring stage, short MMAs) but need more waves; wide
+// tiles reuse each A stage over more columns but run longer per wave.  Row
+// tails count as whole 128-row tiles, so an M with a small M % 128 pays for
+// the padding it creates (the audit's tail-tile rule, restated as waves over
+// 148 SMs); the narrow N = 96 projections favour spreading tiles over SMs.
 // Groups packed per tile of width bn: a tile holds whole groups when N
 // divides bn and is a multiple of 16 (so no 16-column chunk straddles two
 // groups); otherwise 1 (a group spans ceil(N / bn) tiles).
@@ -519,22 +519,17 @@ int64_t n_slots(int bn, int N, int G, int P) {
 
 int select_tile_grouped(int M, int N, int K, int G, int sms) {
     if (M < 1 || N < 1 || K < 1 || G < 1 || sms < 1) return -1;
-    const double eff[kNumTiles] = {0.30, 0.55, 0.70, 0.80, 0.88, 0.92};
-    const double per_sm_flops_us = 1.6e15 / 148.0 * 1e-6;   // dense f16 per SM per microsecond
-    const double hbm_bytes_us = 6.5e6;                       // ~6.5 TB/s in bytes per microsecond
+    // ns per k-block of one tile, for BN = 32, 64, 96, 128, 192, 256.
+    const double kb_ns[kNumTiles] = {175.0, 193.0, 262.0, 262.0, 338.0, 438.0};
+    const int64_t nkb = (K + BK - 1) / BK;
     int best = -1;
     double best_t = 1e300;
     for (int t = 0; t < kNumTiles; ++t) {
         const int bn = kTiles[t].bn;
         const int P = pack_factor(bn, N, G);
         const int64_t tiles = (int64_t)((M + BM - 1) / BM) * n_slots(bn, N, G, P);
-        const int64_t active = std::min<int64_t>(tiles, sms);
         const int64_t waves = (tiles + sms - 1) / sms;
-        const double kpad = (double)((K + BK - 1) / BK * BK);
-        const double tile_us = 2.0 * BM * bn * kpad / (per_sm_flops_us * eff[t]) + 0.3;
-        const double sm_bw = std::min(1.0e5, hbm_bytes_us / (double)active);
-        const double stream_us = (BM + bn) * kpad * 2.0 / sm_bw;
-        const double t_est = (double)waves * std::max(tile_us, stream_us);
+        const double t_est = (double)waves * (double)nkb * kb_ns[t];
         if (t_est < best_t * 0.999) {
             best_t = t_est;
             best = t;
