@@ -518,23 +518,35 @@ def run_e2e(rb, args, world, device, fused=True):
     import torch
     mr = rb.mr
     flags = 0 if args.no_pdl else mr.MR_GEMV_PDL
-    a_host = torch.from_numpy(rb.a16.view(np.int16)).pin_memory()
-    idx_host = {m: torch.empty((m, TOPK), dtype=torch.int32).pin_memory() for m in WINDOWS}
-    val_host = {m: torch.empty((m, TOPK), dtype=torch.float32).pin_memory() for m in WINDOWS}
-    a_dev = {m: torch.empty((m, K_ROUTER), dtype=torch.int16, device=device) for m in WINDOWS}
+    # The step's rows for every window, stacked (1 + 2 + 4 + 8 + 16 = 31 rows):
+    # one host -> device copy of all inputs and one device -> host copy each of
+    # the indices and values per step, with each window's calls on its slice.
+    rows = step_rows()
+    offs, o = {}, 0
+    for m in WINDOWS:
+        offs[m] = o
+        o += m
+    a_rows = np.concatenate([rb.a16[:m] for m in WINDOWS]).view(np.int16)
+    a_host = torch.from_numpy(a_rows).pin_memory()
+    idx_host = torch.empty((rows, TOPK), dtype=torch.int32).pin_memory()
+    val_host = torch.empty((rows, TOPK), dtype=torch.float32).pin_memory()
+    a_dev = torch.empty((rows, K_ROUTER), dtype=torch.int16, device=device)
+    idx_dev = torch.empty((rows, TOPK), dtype=torch.int32, device=device)
+    val_dev = torch.empty((rows, TOPK), dtype=torch.float32, device=device)
     steps = max(1, min(args.steps, 2000))
 
     def one_step():
+        a_dev.copy_(a_host, non_blocking=True)
         for m in WINDOWS:
-            a_dev[m].copy_(a_host[:m], non_blocking=True)
+            sl = slice(offs[m], offs[m] + m)
             if fused:
-                mr.router_gemv_topk(a_dev[m], rb._next_w(), TOPK, rb.idx[m], rb.val[m], workspace=rb.ws,
+                mr.router_gemv_topk(a_dev[sl], rb._next_w(), TOPK, idx_dev[sl], val_dev[sl], workspace=rb.ws,
                                     flags=flags)
             else:
-                mr.mrgemv_bf16(a_dev[m], rb._next_w(), rb.C[m], flags=flags)
-                mr.router_topk(rb.C[m], TOPK, rb.idx[m], rb.val[m])
-            idx_host[m].copy_(rb.idx[m], non_blocking=True)
-            val_host[m].copy_(rb.val[m], non_blocking=True)
+                mr.mrgemv_bf16(a_dev[sl], rb._next_w(), rb.C[m], flags=flags)
+                mr.router_topk(rb.C[m], TOPK, idx_dev[sl], val_dev[sl])
+        idx_host.copy_(idx_dev, non_blocking=True)
+        val_host.copy_(val_dev, non_blocking=True)
 
     with torch.cuda.stream(rb.stream):
         for _ in range(3):
