@@ -43,7 +43,15 @@
 namespace mr {
 namespace gemv {
 
-constexpr int kMaxWarps = 8;
+// Warps per CTA at most, and the unroll of the k loop, per (rows, columns per
+// group).  16 warps (512 threads, so at most 128 registers each) give the
+// FMA-bound shapes twice the warps to hide shared-memory and FMA latency; the
+// 8-row, 8-column kernel needs ~230 registers for its accumulators and W
+// operands and keeps 8 warps.  The 8- and 16-row kernels fit 128 registers
+// only without unrolling the k loop.  None of this changes an output's
+// arithmetic: a lane's chain and the reduction order are fixed by k.
+__host__ __device__ constexpr int warps_max(int MB, int CG) { return (MB == 8 && CG == 8) ? 8 : 16; }
+__host__ __device__ constexpr int q_unroll(int MB, int CG) { return (MB >= 8 && warps_max(MB, CG) == 16) ? 1 : 2; }
 constexpr int kMaxRows = 16;
 
 struct Params {
@@ -197,7 +205,7 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
 #pragma unroll
         for (int j = 0; j < NC; ++j) acc[rp][j] = 0ull;
 
-#pragma unroll 2
+#pragma unroll (q_unroll(MB, CGMAX))
     for (int q = q_begin + lane; q < q_end; q += 32) {
         uint64_t wd[4][NC];  // (w, w) for element e of the chunk, column j
 #pragma unroll
@@ -276,7 +284,7 @@ __device__ __forceinline__ bool run_group(const Params &p, const Smem &sm, int g
 }
 
 template <int MB, int CG, bool FUSED>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const Params p) {
+__global__ void __launch_bounds__(warps_max(MB, CG) * 32, 1) gemv_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
 
     const int tid = threadIdx.x;
@@ -585,11 +593,11 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     pl.KW = k_warps(k);
     pl.G = std::min(sms, n);
     const int ng_max = ng_max_of(n, pl.G, pl.CG);
-    const int cwg0 = std::max(1, std::min(ng_max, kMaxWarps / pl.KW));
+    const int cwg0 = std::max(1, std::min(ng_max, warps_max(pl.MB, pl.CG) / pl.KW));
     pl.a_bytes = (uint32_t)(((size_t)pl.MB * k * 2 + 127) / 128 * 128);
     pl.slot_bytes = (uint32_t)pl.CG * (uint32_t)k * 2u;
     const size_t red_bytes = red_floats(pl.KW, ng_max, pl.MB, pl.CG) * sizeof(float);
-    const size_t topk_bytes = fused ? (size_t)kMaxWarps * 64 * 8 : 0;
+    const size_t topk_bytes = fused ? (size_t)warps_max(pl.MB, pl.CG) * 64 * 8 : 0;
     const size_t fixed = topk_bytes + pl.a_bytes + 24 * (size_t)ng_max + 48 + red_bytes + 64;
     const size_t pdl_budget = 110 * 1024;
     const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, (size_t)optin) : (size_t)optin;
