@@ -14,8 +14,8 @@
 //    are loaded by TMA (no multicast) into a ring of shared-memory stages,
 //    full/empty mbarriers between the producers and the MMA thread.  Each
 //    ring step (barrier wait, TMA or MMA issue, commit) costs a few hundred
-//    cycles of latency: two producer warps alternate stages, and the narrow
-//    tiles, whose MMAs are short, put two k-blocks in a stage;
+//    cycles of latency: two producer warps alternate stages, and the tiles
+//    up to BN = 128, whose MMAs are short, put two k-blocks in a stage;
 //  * tcgen05.mma.cta_group::1.kind::f16 with M = 128, N = BN, K = 16,
 //    accumulating fp32 in tensor memory.  Every tile runs the same sequence of
 //    K steps (16 at a time, ascending, zero padding past K), with no split-K
@@ -56,12 +56,14 @@ struct TileDesc {
     const char *name;
 };
 
-// Narrow tiles take two k-blocks per ring stage: their MMAs are short (the
-// operand reads from shared memory bound them), so one barrier round trip and
-// one commit per k-block would leave the tensor pipe idle between stages.
+// Tiles up to BN = 128 take two k-blocks per ring stage: their MMAs are short
+// (the operand reads from shared memory bound them), so one barrier round trip
+// and one commit per k-block would leave the tensor pipe idle between stages.
+// The wider tiles keep one, since two 40-48 KB k-blocks per stage would leave
+// only two stages in flight.
 constexpr TileDesc kTiles[] = {
-    {32, 8, 32, 2, "128x32"},   {64, 8, 64, 2, "128x64"},   {96, 7, 128, 1, "128x96"},
-    {128, 6, 128, 1, "128x128"}, {192, 5, 256, 1, "128x192"}, {256, 4, 256, 1, "128x256"},
+    {32, 8, 32, 2, "128x32"},   {64, 8, 64, 2, "128x64"},   {96, 7, 128, 2, "128x96"},
+    {128, 6, 128, 2, "128x128"}, {192, 5, 256, 1, "128x192"}, {256, 4, 256, 1, "128x256"},
 };
 constexpr int kNumTiles = sizeof(kTiles) / sizeof(kTiles[0]);
 
@@ -520,7 +522,7 @@ int64_t n_slots(int bn, int N, int G, int P) {
 int select_tile_grouped(int M, int N, int K, int G, int sms) {
     if (M < 1 || N < 1 || K < 1 || G < 1 || sms < 1) return -1;
     // ns per k-block of one tile, for BN = 32, 64, 96, 128, 192, 256.
-    const double kb_ns[kNumTiles] = {175.0, 193.0, 262.0, 262.0, 338.0, 438.0};
+    const double kb_ns[kNumTiles] = {175.0, 193.0, 225.0, 254.0, 338.0, 438.0};
     const int64_t nkb = (K + BK - 1) / BK;
     int best = -1;
     double best_t = 1e300;
