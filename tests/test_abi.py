@@ -122,7 +122,7 @@ def test_selector_tail_rule_and_measured_choices():
         for rt in (2, 5, 11, 16):
             picks = {mr.gemm_f16_select_tile(M, N, 2560) for M in (128 * (rt - 1) + 1, 128 * rt - 64, 128 * rt)}
             assert len(picks) == 1, (N, rt, picks)
-    measured_best = {(150, 512): "128x32", (1300, 512): "128x64", (1983, 1664): "128x192",
+    measured_best = {(306, 640): "128x32", (1300, 512): "128x64", (1983, 1664): "128x192",
                      (1300, 4096): "128x192", (306, 6144): "128x128", (2048, 4096): "128x256",
                      (700, 6144): "128x256", (448, 4096): "128x128", (150, 4096): "128x64",
                      (1983, 1152): "128x128", (448, 6144): "128x192"}
