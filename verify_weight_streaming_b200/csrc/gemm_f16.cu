@@ -290,9 +290,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // Warps 0 and 1 run their loops as whole warps (every lane waits on the
-    // same barrier) and let lane 0 issue: a lone lane spinning in try_wait
-    // beside warp-mates parked elsewhere can stall for the suspend limit.
+    // The producer and MMA warps run their loops as whole warps (every lane
+    // waits on the same barrier) and let one lane issue: a lone lane spinning
+    // in try_wait beside warp-mates parked elsewhere can stall for the
+    // suspend limit.
     if (warp == 0 || warp == 6) {
         // Producers: stage `it` counts across tiles, so slots and phases
         // continue from one tile to the next.
