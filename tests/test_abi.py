@@ -193,3 +193,41 @@ def test_gemm_raster_validation():
     assert g(A16, 64, A16, 64, A16, 32, 4, 32, 64, 0, 0, -1, -1, None) == mr.MR_ERR_INVALID_ARG
     assert g(A16, 64, A16, 64, A16, 32, 4, 32, 64, 0, 0, -1, 65, None) == mr.MR_ERR_INVALID_ARG
     assert g(A16, 64, A16, 64, A16, 32, 4, 32, 64, 0, 0, -1, 8, None) == mr.MR_ERR_CUDA  # valid; no device
+
+
+def test_header_compiles_as_c99_and_links_from_c(tmp_path):
+    """The boundary is a C ABI: the header compiles as strict C99 and a C
+    program links against the library and gets the documented status codes
+    from host-side validation (no device needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "mrgemm.h"
+int main(void) {
+    int32_t out[8];
+    int32_t idx[10];
+    printf("%s\n", mr_version());
+    printf("%d\n", (int)mrgemv_bf16(NULL, 64, NULL, 64, NULL, 32, 4, 32, 64, NULL));
+    printf("%d\n", (int)mrgemv_bf16_plan(17, 512, 2560, 0, 148, 232448, out));
+    printf("%d\n", (int)router_topk(NULL, 512, 1, 512, 10, idx, NULL, 10, NULL));
+    printf("%d\n", (int)gemm_f16_select_tile(2048, 6144, 2560));
+    printf("%s\n", mr_status_str(MR_ERR_MISALIGNED));
+    return 0;
+}
+''')
+    libdir = os.path.dirname(mr.LIB)
+    exe = tmp_path / "abi"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.dirname(HEADER), str(src),
+                    "-L", libdir, "-lmrgemm", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    lines = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    assert "sm_100a" in lines[0]
+    assert int(lines[1]) == mr.MR_ERR_INVALID_ARG
+    assert int(lines[2]) == mr.MR_ERR_UNSUPPORTED
+    assert int(lines[3]) == mr.MR_ERR_INVALID_ARG
+    assert mr.gemm_f16_tile_name(int(lines[4])) == "128x256"
+    assert lines[5] == "MR_ERR_MISALIGNED"
