@@ -85,7 +85,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
-// ---- bulk copies (non-tensor, no multicast) -------------------------------
+// ---- bulk copies (non-tensor, into the issuing CTA only) ------------------
 
 // Global -> shared bulk copy of `bytes` (multiple of 16, both addresses
 // 16-byte aligned) whose completion is counted on `bar` as tx bytes.

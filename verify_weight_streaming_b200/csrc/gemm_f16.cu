@@ -11,7 +11,7 @@
 //    (tcgen05.ld) and store the tile.  Two accumulator buffers in tensor
 //    memory let one tile's epilogue run under the next tile's MMAs;
 //  * A and Wt k-blocks of 64 K-elements (one 128-byte swizzle atom per row)
-//    are loaded by TMA (no multicast) into a ring of shared-memory stages,
+//    are loaded by TMA, each CTA for itself, into a ring of shared-memory stages,
 //    full/empty mbarriers between the producers and the MMA thread.  Each
 //    ring step (barrier wait, TMA or MMA issue, commit) costs a few hundred
 //    cycles of latency: two producer warps alternate stages, and the tiles

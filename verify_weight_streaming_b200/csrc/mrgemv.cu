@@ -11,7 +11,7 @@
 //    [b*n/G, (b+1)*n/G) of Wt, i.e. a contiguous run of weight rows.
 //  * The block streams through a ring of shared-memory slots, one column group
 //    (up to CG columns x k) per slot, with cp.async.bulk global->shared copies
-//    counted on an mbarrier (no tensor map, no multicast).  Group g is consumed
+//    counted on an mbarrier (no tensor map; each copy lands in its own CTA).  Group g is consumed
 //    by column warp g % CWG from slot g % S; when slots are refilled, S is a
 //    multiple of CWG, so each slot has a single consumer warp that waits for
 //    the slot's successive uses in order.  The first slots are
