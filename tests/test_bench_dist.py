@@ -49,3 +49,13 @@ def test_two_rank_timing_is_max_over_ranks():
     assert [o[1] for o in out] == [15.0, 15.0]
     assert [o[2] for o in out] == [(2, 0, 0), (2, 1, 1)]
     assert out[1][3] is None  # only rank 0 runs and prints the reference arm
+
+
+def test_source_hash_ignores_comments_only():
+    """A recorded ncu traffic figure stays valid across comment edits and is
+    dropped by any code edit."""
+    import bench
+    code = "int f(int x) {\n    return x + 1;  // one\n}\n/* block\n comment */\n"
+    assert bench._code_only(code) == bench._code_only(code.replace("// one", "// two").replace("block", "other"))
+    assert bench._code_only(code) != bench._code_only(code.replace("x + 1", "x + 2"))
+    assert bench.recorded_traffic("gemv_router") is not None
