@@ -58,4 +58,3 @@ def test_source_hash_ignores_comments_only():
     code = "int f(int x) {\n    return x + 1;  // one\n}\n/* block\n comment */\n"
     assert bench._code_only(code) == bench._code_only(code.replace("// one", "// two").replace("block", "other"))
     assert bench._code_only(code) != bench._code_only(code.replace("x + 1", "x + 2"))
-    assert bench.recorded_traffic("gemv_router") is not None
