@@ -179,3 +179,11 @@ def test_back_to_back_pdl_launches_in_a_graph():
         c = host(C)
         check(c, a, w)
         assert np.array_equal(c.view(np.uint32), e.view(np.uint32))
+
+
+def test_binding_launches_on_the_current_torch_stream():
+    s = torch.cuda.Stream()
+    assert mr._current_stream_handle() == torch.cuda.current_stream().cuda_stream
+    with torch.cuda.stream(s):
+        assert mr._current_stream_handle() == s.cuda_stream
+    assert mr._current_stream_handle() == torch.cuda.current_stream().cuda_stream

@@ -96,10 +96,26 @@ def _check(status: int, call: str) -> None:
         raise MrError(status, call)
 
 
+_current_raw_stream = None
+
+
+def _current_stream_handle() -> int:
+    """The current CUDA stream of the current device, as torch sees it."""
+    global _current_raw_stream
+    if _current_raw_stream is None:
+        import torch
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        dev = getattr(torch._C, "_cuda_getDevice", None)
+        if raw is not None and dev is not None:
+            _current_raw_stream = lambda: raw(dev())  # noqa: E731  (one C++ call each, per launch)
+        else:
+            _current_raw_stream = lambda: torch.cuda.current_stream().cuda_stream  # noqa: E731
+    return _current_raw_stream()
+
+
 def _stream(stream):
     if stream is None:
-        import torch
-        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        return ctypes.c_void_p(_current_stream_handle())
     if isinstance(stream, int):
         return ctypes.c_void_p(stream)
     return ctypes.c_void_p(stream.cuda_stream)
