@@ -122,9 +122,11 @@ def _stream(stream):
 
 
 def _rows(t, name):
-    if t.dim() != 2 or t.stride(1) != 1:
+    st = t.stride()
+    if len(st) != 2 or st[1] != 1:
         raise ValueError(f"{name} must be a 2-D tensor with unit column stride")
-    return t.shape[0], t.shape[1], t.stride(0)
+    sh = t.shape
+    return sh[0], sh[1], st[0]
 
 
 def _dtype_code(t) -> int:
