@@ -544,16 +544,19 @@ def run_e2e(rb, args, world, device, fused=True):
     val_dev = torch.empty((rows, TOPK), dtype=torch.float32, device=device)
     steps = max(1, min(args.steps, 2000))
 
+    # Each window's views of the stacked buffers, made once.
+    views = {m: (a_dev[offs[m]:offs[m] + m], idx_dev[offs[m]:offs[m] + m], val_dev[offs[m]:offs[m] + m])
+             for m in WINDOWS}
+
     def one_step():
         a_dev.copy_(a_host, non_blocking=True)
         for m in WINDOWS:
-            sl = slice(offs[m], offs[m] + m)
+            a_m, idx_m, val_m = views[m]
             if fused:
-                mr.router_gemv_topk(a_dev[sl], rb._next_w(), TOPK, idx_dev[sl], val_dev[sl], workspace=rb.ws,
-                                    flags=flags)
+                mr.router_gemv_topk(a_m, rb._next_w(), TOPK, idx_m, val_m, workspace=rb.ws, flags=flags)
             else:
-                mr.mrgemv_bf16(a_dev[sl], rb._next_w(), rb.C[m], flags=flags)
-                mr.router_topk(rb.C[m], TOPK, idx_dev[sl], val_dev[sl])
+                mr.mrgemv_bf16(a_m, rb._next_w(), rb.C[m], flags=flags)
+                mr.router_topk(rb.C[m], TOPK, idx_m, val_m)
         idx_host.copy_(idx_dev, non_blocking=True)
         val_host.copy_(val_dev, non_blocking=True)
 
