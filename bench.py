@@ -528,8 +528,8 @@ def run_e2e(rb, args, world, device, fused=True):
     mr = rb.mr
     flags = 0 if args.no_pdl else mr.MR_GEMV_PDL
     # The step's rows for every window, stacked (1 + 2 + 4 + 8 + 16 = 31 rows):
-    # one host -> device copy of all inputs and one device -> host copy each of
-    # the indices and values per step, with each window's calls on its slice.
+    # one host -> device copy of all inputs and one device -> host copy of the
+    # results per step, with each window's calls on its slice.
     rows = step_rows()
     offs, o = {}, 0
     for m in WINDOWS:
@@ -537,11 +537,13 @@ def run_e2e(rb, args, world, device, fused=True):
         o += m
     a_rows = np.concatenate([rb.a16[:m] for m in WINDOWS]).view(np.int16)
     a_host = torch.from_numpy(a_rows).pin_memory()
-    idx_host = torch.empty((rows, TOPK), dtype=torch.int32).pin_memory()
-    val_host = torch.empty((rows, TOPK), dtype=torch.float32).pin_memory()
+    # Indices and values of a row side by side in one buffer (the API takes
+    # them with a common row stride), so one copy brings both back.
+    out_host = torch.empty((rows, 2 * TOPK), dtype=torch.int32).pin_memory()
     a_dev = torch.empty((rows, K_ROUTER), dtype=torch.int16, device=device)
-    idx_dev = torch.empty((rows, TOPK), dtype=torch.int32, device=device)
-    val_dev = torch.empty((rows, TOPK), dtype=torch.float32, device=device)
+    out_dev = torch.empty((rows, 2 * TOPK), dtype=torch.int32, device=device)
+    idx_dev = out_dev[:, :TOPK]
+    val_dev = out_dev.view(torch.float32)[:, TOPK:]
     steps = max(1, min(args.steps, 2000))
 
     # Each window's views of the stacked buffers, made once.
@@ -557,8 +559,7 @@ def run_e2e(rb, args, world, device, fused=True):
             else:
                 mr.mrgemv_bf16(a_m, rb._next_w(), rb.C[m], flags=flags)
                 mr.router_topk(rb.C[m], TOPK, idx_m, val_m)
-        idx_host.copy_(idx_dev, non_blocking=True)
-        val_host.copy_(val_dev, non_blocking=True)
+        out_host.copy_(out_dev, non_blocking=True)
 
     with torch.cuda.stream(rb.stream):
         for _ in range(3):
@@ -573,6 +574,11 @@ def run_e2e(rb, args, world, device, fused=True):
         end.record(rb.stream)
     torch.cuda.synchronize()
     us = max_over_ranks(start.elapsed_time(end) * 1e3, world, device)
+    # The last step's results, as they reached the host: valid indices, and
+    # values in the top-k's order (non-increasing along each row).
+    got_idx = out_host[:, :TOPK].numpy()
+    got_val = out_host.view(torch.float32)[:, TOPK:].numpy()
+    results_ok = bool(((got_idx >= 0) & (got_idx < N_ROUTER)).all() and (np.diff(got_val, axis=1) <= 0).all())
     # The same steps with their public-API calls captured into CUDA graphs,
     # one graph per step on its own slice of the weight pool (weights still
     # from HBM).  The host copies are graph nodes, so every replay moves the
@@ -615,6 +621,7 @@ def run_e2e(rb, args, world, device, fused=True):
             "api": ("router_gemv_topk" if fused else "mrgemv_bf16 + router_topk")
                    + " (verify_weight_streaming_b200), pinned host buffers",
             "graph_value": (graph_us / (steps * step_rows() * world)) if graph_us is not None else None,
+            "results_ok": results_ok,
             "graph_note": "same calls and host copies, captured once into a CUDA graph and replayed"}
 
 
