@@ -2,10 +2,12 @@
 
 One step = one pass of the router hot path over one batch: for each window
 size m in (1, 2, 4, 8, 16), A[m,2560] bf16 x W_r[2560,512] bf16 -> fp32 logits
-(weight streamed once) -> per-row top-10, in one fused launch per window
-(router_gemv_topk).  That is 31 rows and 5 kernel launches per step; the
-two-launch form (mrgemv_bf16 then router_topk) is timed alongside.  The weight comes from a rotating pool
-of copies larger than twice the L2, so every launch reads it from HBM.
+(weight streamed once) -> per-row top-10.  That is 31 rows per step.  Both
+public forms are timed over the same K steps: one fused launch per window
+(router_gemv_topk) and two launches per window (mrgemv_bf16 then
+router_topk); the faster is the reported value.  The weight comes from a
+rotating pool of copies larger than twice the L2, so every launch reads it
+from HBM.
 
 Printed (rank 0, one JSON line): us_per_row over the whole step (lower is
 better), the per-m curve (us_per_row, GB/s, the batching speedup
