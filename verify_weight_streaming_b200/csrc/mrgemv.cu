@@ -11,12 +11,14 @@
 //    [b*n/G, (b+1)*n/G) of Wt, i.e. a contiguous run of weight rows.
 //  * The block streams through a ring of shared-memory slots, one column group
 //    (up to CG columns x k) per slot, with cp.async.bulk global->shared copies
-//    counted on an mbarrier (no tensor map; each copy lands in its own CTA).  Group g is consumed
-//    by column warp g % CWG from slot g % S; when slots are refilled, S is a
-//    multiple of CWG, so each slot has a single consumer warp that waits for
-//    the slot's successive uses in order.  The first slots are
-//    requested before griddepcontrol.wait, so under programmatic dependent
-//    launch the weight stream overlaps the previous kernel.
+//    counted on an mbarrier (no tensor map; each copy lands in its own CTA).
+//    Group g is consumed by column warp g % CWG from slot g % S; when slots
+//    are refilled, S is a multiple of CWG, so each slot has a single consumer
+//    warp that waits for the slot's successive uses in order.  The first slots
+//    are requested before griddepcontrol.wait, so under programmatic
+//    dependent launch the weight stream overlaps the previous kernel.
+//  * KW x CWG warps per CTA, at most 16 (8 for the 8-row, 8-column kernel).
+//    More warps than k-slices work on separate column groups in parallel.
 //  * A (m rows, bf16) is staged once in shared memory by a bulk copy issued
 //    after the grid-dependency wait, right after the first weight chunk and
 //    before the others (copies from one CTA are served roughly in order, so A
