@@ -30,6 +30,8 @@ MUTANTS = {
     "bf16_ties_away": ("lower > 0x8000u || (lower == 0x8000u && (upper & 1u))", "lower >= 0x8000u"),
     "bf16_truncate": ("upper += 1u;", "upper += 0u;"),
     "sigmoid_sign": ("1.0 / (1.0 + exp(-x))", "1.0 / (1.0 + exp(x))"),
+    "float_accumulator": ("double acc = 0.0, mag = 0.0;", "float acc = 0.0f, mag = 0.0f;"),
+    "descending_k": ("for (int64_t p = 0; p < k; ++p) {", "for (int64_t p = k - 1; p >= 0; --p) {"),
 }
 
 

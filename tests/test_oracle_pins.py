@@ -142,6 +142,37 @@ def pin_statistics(orc):
     assert abs(c.mean()) < 0.05
 
 
+def _cancellation_cases():
+    """Cases of tests/golden/cancellation.txt: (name, fmt, A bits, Wt bits, C, S)."""
+    out = []
+    with open(os.path.join(GOLDEN, "cancellation.txt")) as f:
+        for line in f:
+            tok = line.split("#")[0].split()
+            if not tok:
+                continue
+            name, fmt, rest = tok[0], tok[1], tok[2:]
+            c, s = float(rest[-2]), float(int(rest[-1]))
+            bits = []
+            for t in rest[:-2]:
+                h, _, rep = t.partition("*")
+                bits += [int(h, 16)] * (int(rep) if rep else 1)
+            k = len(bits) // 2
+            a = np.array(bits[:k], dtype=np.uint16).reshape(1, k)
+            w = np.array(bits[k:], dtype=np.uint16).reshape(1, k)
+            out.append((name, fmt, a, w, c, s))
+    return out
+
+
+def pin_fp64_ascending_accumulation(orc):
+    """Cancellation cases worked by hand: they hold only for a binary64 sum in ascending p."""
+    cases = _cancellation_cases()
+    assert len(cases) == 5
+    for name, fmt, a, w, c_ref, s_ref in cases:
+        c, s = orc.matmul(a, fmt, w, fmt)
+        assert c[0, 0] == c_ref, (name, fmt, c[0, 0], c_ref)
+        assert s[0, 0] == s_ref, (name, fmt, s[0, 0], s_ref)
+
+
 def _brute_topk(row, k):
     """k rounds of a linear scan for the best remaining element (selection, not sort)."""
     taken = np.zeros(row.size, dtype=bool)
@@ -245,7 +276,8 @@ def pin_sigmoid(orc):
 
 ALL_PINS = [pin_decode_bf16, pin_decode_f16, pin_integer_bruteforce, pin_mixed_formats,
             pin_worked_example, pin_identity_and_permutation, pin_closed_forms,
-            pin_invariants, pin_statistics, pin_topk_bruteforce, pin_topk_library_sort,
+            pin_invariants, pin_statistics, pin_fp64_ascending_accumulation, pin_topk_bruteforce,
+            pin_topk_library_sort,
             pin_ulp, pin_cast_bf16, pin_sigmoid]
 
 

@@ -69,3 +69,53 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     st = mr.lib.router_gemv_topk_noalloc(A.data_ptr(), 64, W.data_ptr(), 64, None, n, 16, n, 64, 10,
                                          idx.data_ptr(), None, 10, 0, None)
     assert st == mr.MR_ERR_UNSUPPORTED
+
+
+def _graph_nodes(graph) -> int:
+    """Nodes of a captured (kept) torch CUDA graph, counted by the driver."""
+    n = ctypes.c_size_t(0)
+    cuda = ctypes.CDLL("libcuda.so.1")
+    cuda.cuGraphGetNodes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_size_t)]
+    assert cuda.cuGraphGetNodes(ctypes.c_void_p(graph.raw_cuda_graph()), None, ctypes.byref(n)) == 0
+    return n.value
+
+
+def test_noalloc_invalid_call_puts_nothing_on_the_stream():
+    """Every argument is checked before the ticket is cleared: an invalid call
+    returns its error and adds no node to a stream being captured."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    m, n, k = 4, 512, 2560
+    A = dev_bits(synth.normal_bits(3200, (m, k), "bf16", 1.0))
+    W = dev_bits(synth.normal_bits(3201, (n, k), "bf16", 0.02))
+    idx = torch.empty((m, 40), dtype=torch.int32, device="cuda")
+    val = torch.empty((m, 40), dtype=torch.float32, device="cuda")
+    x = torch.zeros(4, device="cuda")
+
+    def call(topk=10, idx_ptr=None, kk=k, stream=None):
+        return mr.lib.router_gemv_topk_noalloc(
+            A.data_ptr(), k, W.data_ptr(), k, None, n, m, n, kk, topk,
+            idx.data_ptr() if idx_ptr is None else idx_ptr, val.data_ptr(), 40, 0, stream)
+
+    # A valid call outside capture: the first call on a device looks up the array.
+    assert call() == mr.MR_OK
+    torch.cuda.synchronize()
+    bad = [(dict(topk=0), mr.MR_ERR_INVALID_ARG), (dict(topk=33), mr.MR_ERR_UNSUPPORTED),
+           (dict(idx_ptr=idx.data_ptr() + 2), mr.MR_ERR_MISALIGNED), (dict(kk=12), mr.MR_ERR_MISALIGNED)]
+
+    def capture(body):
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+        s = torch.cuda.Stream()
+        with torch.cuda.graph(g, stream=s):
+            body(ctypes.c_void_p(s.cuda_stream))
+            x.add_(1.0)
+        return _graph_nodes(g)
+
+    base = capture(lambda s: None)
+    statuses = []
+    bad_nodes = capture(lambda s: statuses.extend(call(stream=s, **kw) for kw, _ in bad))
+    assert statuses == [want for _, want in bad]
+    assert bad_nodes == base
+    # A valid call inside the same kind of capture adds its nodes (memset + kernel).
+    assert capture(lambda s: call(stream=s)) == base + 2
+    assert mr.mr_poll_errors() == 0

@@ -2,6 +2,7 @@
 // (mr_poll_errors) and the bounded-wait self test.
 #include "common.cuh"
 
+#include <condition_variable>
 #include <mutex>
 
 namespace mr_host {
@@ -43,11 +44,14 @@ int max_smem_optin() {
 
 namespace mr {
 
-// Exchange target for mr_poll_errors: the error word is read and cleared in
-// one atomic step on the device, then copied back from here.
-__device__ uint32_t g_error_mailbox = 0;
+// Exchange targets for mr_poll_errors: the error word is read and cleared in
+// one atomic step on the device into a mailbox slot, then copied back from
+// there.  Polls that run at the same time (other threads, other streams) each
+// hold their own slot.
+constexpr int kMailboxes = 64;
+__device__ uint32_t g_error_mailbox[kMailboxes];
 
-__global__ void take_errors_kernel() { g_error_mailbox = atomicExch(&g_error_word, 0u); }
+__global__ void take_errors_kernel(int slot) { g_error_mailbox[slot] = atomicExch(&g_error_word, 0u); }
 
 __global__ void selftest_wait_kernel(uint64_t limit_ns) {
     __shared__ __align__(8) uint64_t bar;
@@ -64,19 +68,52 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
 
 }  // namespace mr
 
+namespace mr_host {
+namespace {
+std::mutex g_mailbox_mutex;
+std::condition_variable g_mailbox_free;
+uint64_t g_mailbox_busy[kMaxDevices] = {};
+
+// A free mailbox slot of `device` (waits while all are taken), or -1.
+int take_mailbox(int device) {
+    if (device < 0 || device >= kMaxDevices) return -1;
+    std::unique_lock<std::mutex> lock(g_mailbox_mutex);
+    g_mailbox_free.wait(lock, [&] { return g_mailbox_busy[device] != ~0ull; });
+    const int slot = __builtin_ctzll(~g_mailbox_busy[device]);
+    g_mailbox_busy[device] |= 1ull << slot;
+    return slot;
+}
+
+void give_mailbox(int device, int slot) {
+    {
+        std::lock_guard<std::mutex> lock(g_mailbox_mutex);
+        g_mailbox_busy[device] &= ~(1ull << slot);
+    }
+    g_mailbox_free.notify_one();
+}
+}  // namespace
+}  // namespace mr_host
+
 extern "C" mr_status mr_poll_errors(void *stream, uint32_t *device_flags) {
+    static_assert(mr::kMailboxes == 64, "one bit of the busy mask per mailbox");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess) return MR_ERR_CUDA;
+    const int slot = mr_host::take_mailbox(device);
+    if (slot < 0) return MR_ERR_CUDA;
+    mr_status st = MR_OK;
+    uint32_t flags = 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(1);
     cfg.stream = s;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, mr::take_errors_kernel);
-    if (e != cudaSuccess) return MR_ERR_CUDA;
-    uint32_t flags = 0;
-    e = cudaMemcpyFromSymbolAsync(&flags, mr::g_error_mailbox, sizeof(flags), 0, cudaMemcpyDeviceToHost, s);
-    if (e != cudaSuccess) return MR_ERR_CUDA;
-    e = cudaStreamSynchronize(s);
-    if (e != cudaSuccess) return MR_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, mr::take_errors_kernel, slot) != cudaSuccess ||
+        cudaMemcpyFromSymbolAsync(&flags, mr::g_error_mailbox, sizeof(flags), sizeof(uint32_t) * (size_t)slot,
+                                  cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        st = MR_ERR_CUDA;
+    mr_host::give_mailbox(device, slot);
+    if (st != MR_OK) return st;
     if (device_flags) *device_flags = flags;
     return flags ? MR_ERR_TIMEOUT : MR_OK;
 }

@@ -338,6 +338,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         // Descriptors of slot 0; a slot's descriptor adds its byte offset >> 4
         // to the start-address field (shared addresses stay below 2^18).
         const uint64_t adesc0 = sw128_desc(sA), bdesc0 = sw128_desc(sB);
+        // One lane issues every MMA and every commit: tcgen05.commit tracks
+        // only the tcgen05 operations of the thread that issues it.
+        const bool leader = elect_one();
         uint32_t it = 0, ti = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++ti) {
@@ -355,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 if (!ok) break;
                 tc_fence_after();
                 __syncwarp();
-                if (elect_one()) {
+                if (leader) {
                     // K steps of 16 in ascending order: every tile and every
                     // stage grouping issues the same MMA sequence.
 #pragma unroll
@@ -373,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 }
                 __syncwarp();
             }
-            if (ok && lane == 0) mma_commit(smem_u32(&acc_full[b]));
+            if (ok && leader) mma_commit(smem_u32(&acc_full[b]));
             __syncwarp();
         }
     } else {

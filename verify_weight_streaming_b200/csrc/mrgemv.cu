@@ -662,9 +662,11 @@ struct FusedArgs {
     uint32_t *ticket;
 };
 
-// Validate, plan and launch; `fused` adds the router top-k of every row.
-mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *C, int64_t ldc, int32_t m,
-                 int32_t n, int32_t k, uint32_t flags, void *stream, const FusedArgs *fused) {
+// Validate and plan a launch without touching the device or any stream:
+// every argument error is found here, before anything is enqueued.  `fused`
+// adds the router top-k of every row.
+mr_status prepare(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *C, int64_t ldc, int32_t m,
+                  int32_t n, int32_t k, uint32_t flags, const FusedArgs *fused, Params &p, Plan &pl) {
     if (!A || !Wt || !C) return MR_ERR_INVALID_ARG;
     if (m < 1 || n < 1 || k < 1) return MR_ERR_INVALID_ARG;
     if (lda < k || ldw < k || ldc < n) return MR_ERR_INVALID_ARG;
@@ -674,17 +676,13 @@ mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float 
     if (((uintptr_t)A & 15u) || ((uintptr_t)Wt & 15u) || ((uintptr_t)C & 3u)) return MR_ERR_MISALIGNED;
     if (m > kMaxRows) return MR_ERR_UNSUPPORTED;
 
-    int device = 0;
-    cudaError_t e = cudaGetDevice(&device);
-    if (e != cudaSuccess) return mr_host::cuda_status(e);
     const int sms = mr_host::sm_count();
     const int optin = mr_host::max_smem_optin();
     if (sms <= 0 || optin <= 0) return MR_ERR_CUDA;
-    Plan pl;
     const mr_status st = make_plan(m, n, k, flags, sms, optin, pl, fused != nullptr);
     if (st != MR_OK) return st;
 
-    Params p = {};
+    p = Params{};
     p.A = static_cast<const uint16_t *>(A);
     p.lda = lda;
     p.Wt = static_cast<const uint16_t *>(Wt);
@@ -708,7 +706,14 @@ mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float 
         p.ldo = fused->ldo;
         p.ticket = fused->ticket;
     }
+    return MR_OK;
+}
 
+// Launch a prepared plan on `stream`.
+mr_status enqueue(const Params &p, const Plan &pl, uint32_t flags, bool fused, void *stream) {
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) return mr_host::cuda_status(e);
     e = ensure_attributes(device);
     if (e != cudaSuccess) return mr_host::cuda_status(e);
 
@@ -722,9 +727,24 @@ mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = (flags & MR_GEMV_PDL) ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kernel_for(pl.MB, pl.CG, fused != nullptr), p);
+    e = cudaLaunchKernelEx(&cfg, kernel_for(pl.MB, pl.CG, fused), p);
     return mr_host::cuda_status(e);
 }
+
+mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *C, int64_t ldc, int32_t m,
+                 int32_t n, int32_t k, uint32_t flags, void *stream, const FusedArgs *fused) {
+    Params p;
+    Plan pl;
+    const mr_status st = prepare(A, lda, Wt, ldw, C, ldc, m, n, k, flags, fused, p, pl);
+    if (st != MR_OK) return st;
+    return enqueue(p, pl, flags, fused != nullptr, stream);
+}
+
+// The fused router's own checks (top-k arguments and workspace), then the
+// GEMV's; nothing is enqueued.  On success p and pl describe the launch.
+mr_status prepare_router(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *logits, int64_t ldl,
+                         int32_t m, int32_t n, int32_t k, int32_t topk, int32_t *idx, float *val, int64_t ldo,
+                         void *workspace, size_t workspace_bytes, uint32_t flags, Params &p, Plan &pl);
 
 }  // namespace gemv
 }  // namespace mr
@@ -740,10 +760,12 @@ extern "C" size_t router_gemv_topk_workspace_bytes(int32_t m, int32_t n, int32_t
     return MR_ROUTER_TICKET_BYTES + (logits_provided ? 0 : (size_t)m * (size_t)n * sizeof(float));
 }
 
-extern "C" mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *logits,
-                                      int64_t ldl, int32_t m, int32_t n, int32_t k, int32_t topk, int32_t *idx,
-                                      float *val, int64_t ldo, void *workspace, size_t workspace_bytes,
-                                      uint32_t flags, void *stream) {
+namespace mr {
+namespace gemv {
+
+mr_status prepare_router(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *logits, int64_t ldl,
+                         int32_t m, int32_t n, int32_t k, int32_t topk, int32_t *idx, float *val, int64_t ldo,
+                         void *workspace, size_t workspace_bytes, uint32_t flags, Params &p, Plan &pl) {
     if (!idx || !workspace) return MR_ERR_INVALID_ARG;
     if (m < 1 || n < 1 || topk < 1 || topk > n || ldo < topk) return MR_ERR_INVALID_ARG;
     if (topk > 32) return MR_ERR_UNSUPPORTED;
@@ -755,8 +777,23 @@ extern "C" mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt
         C = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + MR_ROUTER_TICKET_BYTES);
         ldc = n;
     }
-    mr::gemv::FusedArgs fa = {topk, idx, val, ldo, static_cast<uint32_t *>(workspace)};
-    return mr::gemv::launch(A, lda, Wt, ldw, C, ldc, m, n, k, flags, stream, &fa);
+    const FusedArgs fa = {topk, idx, val, ldo, static_cast<uint32_t *>(workspace)};
+    return prepare(A, lda, Wt, ldw, C, ldc, m, n, k, flags, &fa, p, pl);
+}
+
+}  // namespace gemv
+}  // namespace mr
+
+extern "C" mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *logits,
+                                      int64_t ldl, int32_t m, int32_t n, int32_t k, int32_t topk, int32_t *idx,
+                                      float *val, int64_t ldo, void *workspace, size_t workspace_bytes,
+                                      uint32_t flags, void *stream) {
+    mr::gemv::Params p;
+    mr::gemv::Plan pl;
+    const mr_status st = mr::gemv::prepare_router(A, lda, Wt, ldw, logits, ldl, m, n, k, topk, idx, val, ldo,
+                                                  workspace, workspace_bytes, flags, p, pl);
+    if (st != MR_OK) return st;
+    return mr::gemv::enqueue(p, pl, flags, true, stream);
 }
 
 extern "C" mr_status mrgemv_bf16(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *C,
@@ -813,11 +850,16 @@ extern "C" mr_status router_gemv_topk_noalloc(const void *A, int64_t lda, const 
     if (m < 1 || n < 1) return MR_ERR_INVALID_ARG;
     if (!logits && (size_t)m * (size_t)n > router_gemv_topk_noalloc_max_logits()) return MR_ERR_UNSUPPORTED;
     void *scratch = nullptr;
-    const mr_status st = mr::gemv::noalloc_scratch(&scratch);
+    mr_status st = mr::gemv::noalloc_scratch(&scratch);
+    if (st != MR_OK) return st;
+    // Every argument is checked before anything is put on the stream.
+    mr::gemv::Params p;
+    mr::gemv::Plan pl;
+    st = mr::gemv::prepare_router(A, lda, Wt, ldw, logits, ldl, m, n, k, topk, idx, val, ldo, scratch,
+                                  mr::gemv::kNoAllocScratchBytes, flags, p, pl);
     if (st != MR_OK) return st;
     // The array keeps whatever the last call left; the ticket must start at zero.
     if (cudaMemsetAsync(scratch, 0, MR_ROUTER_TICKET_BYTES, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return MR_ERR_CUDA;
-    return router_gemv_topk(A, lda, Wt, ldw, logits, ldl, m, n, k, topk, idx, val, ldo, scratch,
-                            mr::gemv::kNoAllocScratchBytes, flags, stream);
+    return mr::gemv::enqueue(p, pl, flags, true, stream);
 }
