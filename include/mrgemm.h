@@ -191,6 +191,45 @@ mr_status router_topk(const float *logits, int64_t ldl, int32_t m, int32_t n,
                       void *stream);
 
 /*
+ * router_topk_ex -- router_topk on a shard of columns: the logits are columns
+ * [index_base, index_base + n) of a wider row, and every index written is
+ * index_base + the column's position in `logits`.  Ties still go to the lower
+ * (global) index.  0 <= index_base and index_base + n <= 2^31 - 1; other
+ * arguments as router_topk (index_base 0 gives exactly router_topk).
+ *
+ * The column split of the router across G devices: each device streams its
+ * own N/G columns of the weight with A replicated, takes the top-k of its
+ * shard, and the G lists are merged (router_topk_merge).  The global top-k
+ * lies in the union of the shards' top-k lists, so the merge is exact.  The
+ * pages place experts and layers on a second card (Strata PR #109,
+ * "Measured" and the release comment); this is that placement for the
+ * router's columns.
+ */
+mr_status router_topk_ex(const float *logits, int64_t ldl, int32_t m, int32_t n,
+                         int32_t topk, int32_t *idx, float *val, int64_t ldo,
+                         int32_t index_base, void *stream);
+
+/*
+ * router_topk_merge -- per-row top-k of candidate (value, index) pairs, under
+ * the order of router_topk: value descending, equal values by index
+ * ascending, -0.0 equal to +0.0, a NaN above +inf.
+ *
+ * Row r has `groups` lists of `per_group` pairs; list g of row r is
+ *   cand_val[g * ld_group + r * ld_row + t], cand_idx[...]   (t < per_group)
+ * (e.g. the [groups][m][per_group] block an all-gather of every shard's
+ * router_topk_ex output yields: ld_row = per_group, ld_group = m * per_group).
+ * The indices of a row must be distinct; an index < 0 marks an empty entry
+ * and is skipped.  idx / val (row stride ldo >= topk) receive the best topk
+ * pairs in rank order, the values bit for bit; where a row has fewer than
+ * topk non-empty pairs the remaining entries are index -1, value NaN.
+ * 1 <= topk <= 32; groups * per_group <= 65536 (MR_ERR_UNSUPPORTED above).
+ */
+mr_status router_topk_merge(const float *cand_val, const int32_t *cand_idx, int32_t m,
+                            int32_t groups, int32_t per_group, int64_t ld_row,
+                            int64_t ld_group, int32_t topk, int32_t *idx, float *val,
+                            int64_t ldo, void *stream);
+
+/*
  * cast_f32_bf16 -- fp32 -> bf16, round to nearest even, for `rows` rows of
  * `cols` values in one launch: the bf16 cast of the verify window's rows in
  * Strata PR #109 ("What": one call, the rows are contiguous), which feeds the

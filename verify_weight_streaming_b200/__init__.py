@@ -21,7 +21,8 @@ MR_GEMV_SIGMOID = 0x2
 MR_DEVERR_GEMV_TIMEOUT, MR_DEVERR_GEMM_TIMEOUT, MR_DEVERR_TOPK_TIMEOUT, MR_DEVERR_SELFTEST = 1, 2, 4, 8
 
 EXPORTS = (
-    "mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
+    "mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_topk_ex",
+    "router_topk_merge", "router_gemv_topk",
     "router_gemv_topk_workspace_bytes", "router_gemv_topk_noalloc", "router_gemv_topk_noalloc_max_logits", "gemm_f16_grouped",
     "gemm_f16_grouped_select_tile", "cast_f32_bf16", "gemm_f16_ex", "gemm_f16", "gemm_f16_num_tiles",
     "gemm_f16_tile_name", "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout",
@@ -50,6 +51,8 @@ def _load() -> ctypes.CDLL:
     L.mrgemv_bf16_ex.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, U32, P]
     L.mrgemv_bf16_plan.argtypes = [I32, I32, I32, U32, I32, I32, P]
     L.router_topk.argtypes = [P, I64, I32, I32, I32, P, P, I64, P]
+    L.router_topk_ex.argtypes = [P, I64, I32, I32, I32, P, P, I64, I32, P]
+    L.router_topk_merge.argtypes = [P, P, I32, I32, I32, I64, I64, I32, P, P, I64, P]
     L.router_gemv_topk.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, I32, P, P, I64, P,
                                    ctypes.c_size_t, U32, P]
     L.router_gemv_topk_workspace_bytes.argtypes = [I32, I32, I32]
@@ -72,7 +75,8 @@ def _load() -> ctypes.CDLL:
     L.mr_status_str.restype = ctypes.c_char_p
     L.mr_version.argtypes = []
     L.mr_version.restype = ctypes.c_char_p
-    for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_gemv_topk",
+    for name in ("mrgemv_bf16", "mrgemv_bf16_ex", "mrgemv_bf16_plan", "router_topk", "router_topk_ex",
+                 "router_topk_merge", "router_gemv_topk",
                  "router_gemv_topk_noalloc", "gemm_f16_grouped", "gemm_f16_grouped_select_tile",
                  "cast_f32_bf16", "gemm_f16_ex", "gemm_f16", "gemm_f16_num_tiles",
                  "gemm_f16_select_tile", "mr_poll_errors", "mr_selftest_wait_timeout"):
@@ -172,6 +176,46 @@ def router_topk(logits, topk: int, idx, val=None, stream=None) -> None:
         vptr = val.data_ptr()
     st = lib.router_topk(logits.data_ptr(), ldl, m, n, topk, idx.data_ptr(), vptr, ldo, _stream(stream))
     _check(st, "router_topk")
+
+
+def router_topk_ex(logits, topk: int, idx, val=None, index_base: int = 0, stream=None) -> None:
+    """router_topk of a shard of columns: indices are written as index_base + column."""
+    m, n, ldl = _rows(logits, "logits")
+    mi, ki, ldo = _rows(idx, "idx")
+    if mi != m or ki < topk:
+        raise ValueError("idx shape mismatch")
+    vptr = None
+    if val is not None:
+        mv, kv, ldv = _rows(val, "val")
+        if mv != m or kv < topk or ldv != ldo:
+            raise ValueError("val must match idx's shape and stride")
+        vptr = val.data_ptr()
+    st = lib.router_topk_ex(logits.data_ptr(), ldl, m, n, topk, idx.data_ptr(), vptr, ldo, index_base,
+                            _stream(stream))
+    _check(st, "router_topk_ex")
+
+
+def router_topk_merge(cand_val, cand_idx, topk: int, idx, val=None, stream=None) -> None:
+    """Per-row top-k of candidate lists laid out [groups, m, per_group] (fp32
+    values, int32 global indices, -1 = empty), e.g. an all-gather of every
+    shard's router_topk_ex output."""
+    if cand_val.dim() != 3 or tuple(cand_idx.shape) != tuple(cand_val.shape):
+        raise ValueError("cand_val and cand_idx must be [groups, m, per_group] of the same shape")
+    if cand_val.stride() != cand_idx.stride() or cand_val.stride(2) != 1:
+        raise ValueError("candidates need a common layout with unit stride in the last dimension")
+    groups, m, per = cand_val.shape
+    mi, ki, ldo = _rows(idx, "idx")
+    if mi != m or ki < topk:
+        raise ValueError("idx shape mismatch")
+    vptr = None
+    if val is not None:
+        mv, kv, ldv = _rows(val, "val")
+        if mv != m or kv < topk or ldv != ldo:
+            raise ValueError("val must match idx's shape and stride")
+        vptr = val.data_ptr()
+    st = lib.router_topk_merge(cand_val.data_ptr(), cand_idx.data_ptr(), m, groups, per, cand_val.stride(1),
+                               cand_val.stride(0), topk, idx.data_ptr(), vptr, ldo, _stream(stream))
+    _check(st, "router_topk_merge")
 
 
 MR_ROUTER_TICKET_BYTES = 256
