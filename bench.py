@@ -388,9 +388,9 @@ def run_gpu(args, world, rank, local):
     clocks_best["other_form"] = clocks[[k for k in clocks if k != best_form][0]]
     del forms
 
-    # ---- per-m curve and the GEMV roofline (back-to-back graph-captured calls)
-    curve = gemv_curve(rb, rb.W, rb.A, K_ROUTER, N_ROUTER, flags, with_router=True)
-    speedup = curve["1"]["us_per_row"] / curve["8"]["us_per_row"]
+    # ---- per-m curves and the GEMV roofline (back-to-back graph-captured calls)
+    curves = gemv_curves(rb, flags, hbm_peak)
+    curve = curves["router"]
     # dominant kernel: the GEMV, averaged over the step's mix of m
     mean_call_us = sum(curve[str(m)]["us_per_call"] for m in WINDOWS) / len(WINDOWS)
     mean_bytes = sum(gemv_bytes(m, N_ROUTER, K_ROUTER) for m in WINDOWS) / len(WINDOWS)
@@ -398,9 +398,10 @@ def run_gpu(args, world, rank, local):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": recorded_traffic("gemv_router"),
                 "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "mrgemv_bf16 (router, m mix 1..16)"}
-    extra_curves = {}
-    if not args.quick:
-        extra_curves = other_gemv_curves(rb, flags)
+    # The FFN and sweep weights (8.7 and 31 MB) are large enough to be HBM-bound:
+    # their fractions of the measured copy bandwidth, m = 1..8, reported apart.
+    roofline["by_shape_m1_to_8"] = {name: {m: curves[name][str(m)]["frac_of_measured_hbm"] for m in (1, 2, 4, 8)}
+                                    for name, _, _ in GEMV_SHAPES}
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(rb, args, world, device, fused=(best_form == "fused"))
@@ -410,9 +411,10 @@ def run_gpu(args, world, rank, local):
     sweep = path_sweep() if not (args.skip_gemm or args.quick) else None
 
     # ---- CPU oracle baseline (rank 0, N=1 only)
-    cpu = None
+    cpu, cpus = None, None
     if rank == 0 and world == 1 and not args.skip_cpu:
         cpu = cpu_baseline(rb)
+        cpus = cpu_baselines()
 
     if rank == 0:
         line = {
@@ -424,8 +426,8 @@ def run_gpu(args, world, rank, local):
             "gpu_launches": args.steps * len(WINDOWS) * (1 if best_form == "fused" else 2),
             "forms_us_per_row": forms_us_per_row,
             "device_errors": errs, "clocks": clocks_best, "roofline": roofline,
-            "curve": {"router": curve, "batching_speedup_m1_over_m8": speedup, **extra_curves},
-            "e2e": e2e, "gemm": gemm, "path_sweep": sweep, "cpu_baseline": cpu,
+            "curve": curves,
+            "e2e": e2e, "gemm": gemm, "path_sweep": sweep, "cpu_baseline": cpu, "cpu_baselines": cpus,
             "pdl": not args.no_pdl,
         }
         print(json.dumps(line), flush=True)
@@ -433,94 +435,124 @@ def run_gpu(args, world, rank, local):
         dist.destroy_process_group()
 
 
-def gemv_curve(rb, pool, A, k, n, flags, launches=None, with_router=False):
-    """us per call / per row and GB/s for each m, from graphs of back-to-back
-    calls over distinct weight copies; plus the per-row-launch mode (m calls
-    of m=1, the unbatched baseline)."""
-    torch, mr = rb.torch, rb.mr
-    launches = launches or min(len(pool), 64)
-    C = torch.empty((16, n), dtype=torch.float32, device=rb.device)
-    cursor = [0]
-
-    def nxt():
-        w = pool[cursor[0] % len(pool)]
-        cursor[0] += 1
-        return w
-
-    def capture(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=rb.stream):
-            fn()
-        return g
-
-    out = {}
-    for m in WINDOWS:
-        def batched():
-            for _ in range(launches):
-                mr.mrgemv_bf16(A[:m], nxt(), C[:m], flags=flags)
-
-        def per_row():
-            for _ in range(max(1, launches // m)):
-                w = nxt()
-                for r in range(m):
-                    mr.mrgemv_bf16(A[r:r + 1], w, C[r:r + 1], flags=flags)
-        with torch.cuda.stream(rb.stream):
-            batched()
-            per_row()
-        torch.cuda.synchronize()
-        g = [capture(batched) for _ in range(2)]
-        rb.time_graphs(g, 2)
-        t = min(rb.time_graphs(g, 8) / (8 * launches) for _ in range(3))
-        gs = [capture(per_row)]
-        rb.time_graphs(gs, 1)
-        t1 = min(rb.time_graphs(gs, 4) / (4 * max(1, launches // m)) for _ in range(2))
-        nbytes = gemv_bytes(m, n, k)
-        out[str(m)] = {"us_per_call": t, "us_per_row": t / m, "GBps": nbytes / (t * 1e3),
-                       "per_row_launch_us_per_row": t1 / m}
-        if with_router:
-            idx = torch.empty((m, TOPK), dtype=torch.int32, device=rb.device)
-            val = torch.empty((m, TOPK), dtype=torch.float32, device=rb.device)
-
-            def fused_calls():
-                for _ in range(launches):
-                    mr.router_gemv_topk(A[:m], nxt(), TOPK, idx, val, workspace=rb.ws, flags=flags)
-
-            def two_calls():
-                for _ in range(launches):
-                    mr.mrgemv_bf16(A[:m], nxt(), C[:m], flags=flags)
-                    mr.router_topk(C[:m], TOPK, idx, val)
-            with torch.cuda.stream(rb.stream):
-                fused_calls()
-                two_calls()
-            torch.cuda.synchronize()
-            gf = [capture(fused_calls)]
-            g2 = [capture(two_calls)]
-            rb.time_graphs(gf, 1)
-            rb.time_graphs(g2, 1)
-            out[str(m)]["router_fused_us_per_window"] = min(rb.time_graphs(gf, 4) / (4 * launches) for _ in range(2))
-            out[str(m)]["router_two_launch_us_per_window"] = min(rb.time_graphs(g2, 4) / (4 * launches) for _ in range(2))
-    return out
+ROUNDS = 5
 
 
-def other_gemv_curves(rb, flags):
-    """The KAT's FFN shape (k=896, n=4864) and the sweep shape (k=2560, n=6144)."""
+def graph_of(torch, stream, fn):
+    """Capture fn() once into a CUDA graph on `stream` (after one eager run)."""
+    with torch.cuda.stream(stream):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    return g
+
+
+def replay_us(torch, stream, graph, reps):
+    """Device time of `reps` back-to-back replays (CUDA events on `stream`), in us."""
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3
+
+
+def interleaved(torch, stream, cases, rounds=ROUNDS):
+    """Time every case once per round, the cases interleaved, for `rounds` rounds.
+
+    A case is (key, graph, units, reps): `units` calls per replay.  Returns
+    {key: {"min": us per unit, "median": us per unit, "samples": [...]}}; min is
+    the primary figure, as in the audit's method (min over interleaved rounds)."""
+    samples = {key: [] for key, _, _, _ in cases}
+    for _ in range(rounds):
+        for key, g, units, reps in cases:
+            samples[key].append(replay_us(torch, stream, g, reps) / (reps * units))
+    return {k: {"min": min(v), "median": statistics.median(v), "samples": v} for k, v in samples.items()}
+
+
+GEMV_SHAPES = (("router", K_ROUTER, N_ROUTER), ("ffn_k896_n4864", 896, 4864), ("sweep_k2560_n6144", 2560, 6144))
+
+
+def gemv_curves(rb, flags, hbm_peak):
+    """us per call and per row, GB/s and the fraction of the measured HBM copy
+    bandwidth for each window size m, on the router, FFN and sweep weights;
+    each from graphs of back-to-back calls over distinct weight copies (more
+    than 2x the L2), min and median over interleaved rounds.  Also the
+    per-row-launch mode (m calls of m = 1, the unbatched baseline) and, on the
+    router, the fused and two-launch router windows."""
     import numpy as np
     import synth
-    torch = rb.torch
-    res = {}
-    for name, k, n, wl in (("ffn_k896_n4864", 896, 4864, synth.WL_GEMV_FFN),
-                           ("sweep_k2560_n6144", 2560, 6144, synth.WL_SWEEP)):
-        a16 = synth.normal_bits(synth.seed_for(wl, 0), (16, k), "bf16", 1.0)
-        w16 = synth.normal_bits(synth.seed_for(wl, 1), (n, k), "bf16", 1.0 / np.sqrt(k))
-        w = torch.from_numpy(w16.view(np.int16)).to(rb.device)
-        copies = max(4, int(math.ceil(2.2 * rb.l2 / w16.nbytes)))
-        pool = [w.clone() for _ in range(copies)]
-        A = torch.from_numpy(a16.view(np.int16)).to(rb.device)
-        c = gemv_curve(rb, pool, A, k, n, flags, launches=max(copies, 16))
-        c["batching_speedup_m1_over_m8"] = c["1"]["us_per_row"] / c["8"]["us_per_row"]
-        res[name] = c
-        del pool, w
-    return res
+    torch, mr = rb.torch, rb.mr
+    stream = rb.stream
+    cases, meta = [], {}
+    keep = []
+    for name, k, n in GEMV_SHAPES:
+        if name == "router":
+            pool, A = rb.W, rb.A
+        else:
+            wl = synth.WL_GEMV_FFN if k == 896 else synth.WL_SWEEP
+            a16 = synth.normal_bits(synth.seed_for(wl, 0), (16, k), "bf16", 1.0)
+            w16 = synth.normal_bits(synth.seed_for(wl, 1), (n, k), "bf16", 1.0 / np.sqrt(k))
+            w = torch.from_numpy(w16.view(np.int16)).to(rb.device)
+            pool = [w.clone() for _ in range(max(4, int(math.ceil(2.2 * rb.l2 / w16.nbytes))))]
+            A = torch.from_numpy(a16.view(np.int16)).to(rb.device)
+        launches = min(len(pool), 64) if name == "router" else max(len(pool), 16)
+        C = torch.empty((16, n), dtype=torch.float32, device=rb.device)
+        keep.append((pool, A, C))
+        for m in WINDOWS:
+            def batched(m=m, pool=pool, A=A, C=C, launches=launches):
+                for i in range(launches):
+                    mr.mrgemv_bf16(A[:m], pool[i % len(pool)], C[:m], flags=flags)
+
+            def per_row(m=m, pool=pool, A=A, C=C, launches=launches):
+                for i in range(max(1, launches // m)):
+                    for r in range(m):
+                        mr.mrgemv_bf16(A[r:r + 1], pool[i % len(pool)], C[r:r + 1], flags=flags)
+            cases.append(((name, m, "batched"), graph_of(torch, stream, batched), launches, 4))
+            cases.append(((name, m, "per_row"), graph_of(torch, stream, per_row), max(1, launches // m), 2))
+            meta[(name, m)] = gemv_bytes(m, n, k)
+            if name == "router":
+                idx = torch.empty((m, TOPK), dtype=torch.int32, device=rb.device)
+                val = torch.empty((m, TOPK), dtype=torch.float32, device=rb.device)
+                keep.append((idx, val))
+
+                def fused(m=m, idx=idx, val=val, launches=launches):
+                    for i in range(launches):
+                        mr.router_gemv_topk(A[:m], pool[i % len(pool)], TOPK, idx, val, workspace=rb.ws, flags=flags)
+
+                def two(m=m, idx=idx, val=val, launches=launches):
+                    for i in range(launches):
+                        mr.mrgemv_bf16(A[:m], pool[i % len(pool)], C[:m], flags=flags)
+                        mr.router_topk(C[:m], TOPK, idx, val)
+                cases.append(((name, m, "fused"), graph_of(torch, stream, fused), launches, 2))
+                cases.append(((name, m, "two_launch"), graph_of(torch, stream, two), launches, 2))
+    t = interleaved(torch, stream, cases)
+    out = {}
+    for name, k, n in GEMV_SHAPES:
+        cur = {}
+        for m in WINDOWS:
+            b = t[(name, m, "batched")]
+            nbytes = meta[(name, m)]
+            row = {"us_per_call": b["min"], "us_per_call_median": b["median"], "us_per_row": b["min"] / m,
+                   "GBps": nbytes / (b["min"] * 1e3), "frac_of_measured_hbm": nbytes / (b["min"] * 1e3) / hbm_peak,
+                   "per_row_launch_us_per_row": t[(name, m, "per_row")]["min"] / m}
+            if name == "router":
+                row["router_fused_us_per_window"] = t[(name, m, "fused")]["min"]
+                row["router_two_launch_us_per_window"] = t[(name, m, "two_launch")]["min"]
+            cur[str(m)] = row
+        cur["batching_speedup_m1_over_m8"] = cur["1"]["us_per_row"] / cur["8"]["us_per_row"]
+        out[name] = cur
+    out["method"] = (f"min (and median) over {ROUNDS} interleaved rounds of graph-replayed back-to-back calls; "
+                     "weights rotated over copies > 2x L2")
+    del cases, keep
+    return out
 
 
 def run_e2e(rb, args, world, device, fused=True):
@@ -640,6 +672,51 @@ def cpu_baseline(rb):
             "sample": f"{steps} router steps (31 rows each: windows m=1,2,4,8,16, 2560x512, top-10)"}
 
 
+def cpu_baselines():
+    """The oracle (plain C, fp64, every host core) beside each of the other
+    workloads, each on a bounded sample (a few seconds of CPU work in all)."""
+    import numpy as np
+    import oracle
+    import synth
+    oracle.default()
+    cores = oracle.num_threads()
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return (time.perf_counter() - t0) * 1e6
+
+    out = {}
+    # FFN GEMV (k = 896, n = 4864), every window size of the workload
+    ffn = {}
+    for m in (1, 2, 4, 8):
+        a, w = synth.gemv_ffn(m)
+        us = timed(lambda: oracle.matmul(a, "bf16", w, "bf16"))
+        ffn[str(m)] = {"us_per_call": us, "us_per_row": us / m, "GFLOPs": 2.0 * m * 4864 * 896 / (us * 1e3)}
+    out["ffn_gemv_k896_n4864"] = {"value": ffn["8"]["us_per_row"], "unit": "us/row", "per_m": ffn,
+                                  "cores": cores, "kind": "oracle", "sample": "full calls, m = 1, 2, 4, 8"}
+    # narrow N = 96 GEMM: one of the 36 projections at M = 512
+    a, w = synth.narrow(512)
+    us = timed(lambda: oracle.matmul(a, "f16", w, "f16"))
+    out["narrow_gemm_n96"] = {"value": us, "unit": "us/call", "GFLOPs": 2.0 * 512 * 96 * 2560 / (us * 1e3),
+                              "cores": cores, "kind": "oracle", "sample": "one 512 x 96 x 2560 call of the 36"}
+    # prompt-chunk GEMM: a tail-tile shape, rows sampled
+    a, w = synth.chunk(306, 1152)
+    us = timed(lambda: oracle.matmul(a[:128], "f16", w, "f16"))
+    out["chunk_gemm_306x1152"] = {"value": us * 306 / 128, "unit": "us/call",
+                                  "GFLOPs": 2.0 * 128 * 1152 * 2560 / (us * 1e3), "cores": cores,
+                                  "kind": "oracle", "sample": "128 of the 306 rows, scaled to the call"}
+    # m-sweep weights (k = 2560, n = 6144): the GEMV at m = 1 and 16 rows of the GEMM side
+    a = synth.normal_bits(synth.seed_for(synth.WL_SWEEP, 0), (16, 2560), "bf16", 1.0)
+    w = synth.normal_bits(synth.seed_for(synth.WL_SWEEP, 1), (6144, 2560), "bf16", 1.0 / np.sqrt(2560))
+    us1 = timed(lambda: oracle.matmul(a[:1], "bf16", w, "bf16"))
+    us16 = timed(lambda: oracle.matmul(a, "bf16", w, "bf16"))
+    out["sweep_k2560_n6144"] = {"value": us16 / 16, "unit": "us/row", "us_per_row_m1": us1,
+                                "GFLOPs": 2.0 * 16 * 6144 * 2560 / (us16 * 1e3), "cores": cores,
+                                "kind": "oracle", "sample": "m = 1 and m = 16 calls"}
+    return out
+
+
 GEMM_M = (150, 192, 306, 448, 700, 1300, 1983, 2048)
 GEMM_N = (512, 640, 1152, 1664, 4096, 6144)
 NARROW_M = (512, 640, 768, 1024, 1983, 2048)
@@ -655,24 +732,8 @@ def run_gemm_sweep(args):
 def _time_calls(torch, calls, reps=3):
     """Graph-capture `calls` (a list of thunks), replay, return us per call (min of reps)."""
     s = torch.cuda.Stream()
-    with torch.cuda.stream(s):
-        for c in calls:
-            c()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=s):
-        for c in calls:
-            c()
-    best = float("inf")
-    for _ in range(reps):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(s):
-            e0.record(s)
-            g.replay()
-            e1.record(s)
-        torch.cuda.synchronize()
-        best = min(best, e0.elapsed_time(e1) * 1e3 / len(calls))
+    g = graph_of(torch, s, lambda: [c() for c in calls])
+    best = min(replay_us(torch, s, g, 1) / len(calls) for _ in range(reps))
     del g
     return best
 
@@ -680,9 +741,10 @@ def _time_calls(torch, calls, reps=3):
 def gemm_sweep(quick=False):
     """TFLOP/s of gemm_f16 (auto tile) on the prompt-chunk and narrow shapes.
 
-    Each shape is timed as graph-replayed back-to-back calls that rotate over
-    weight copies (and A copies) whose total exceeds twice the L2, so operands
-    come from HBM as they would for a chunk's successive projections."""
+    Each shape is a graph of back-to-back calls that rotate over weight copies
+    (and A copies) whose total exceeds twice the L2, so operands come from HBM
+    as they would for a chunk's successive projections.  Every shape is timed
+    once per round, shapes interleaved, over ROUNDS rounds: min and median."""
     import numpy as np
     import torch
     import synth
@@ -691,11 +753,12 @@ def gemm_sweep(quick=False):
     props = torch.cuda.get_device_properties(0)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
     K = 2560
-    out = {"chunk": {}, "narrow": {}}
+    stream = torch.cuda.Stream()
     ms = GEMM_M if not quick else (306, 2048)
     ns = GEMM_N if not quick else (512, 6144)
     a_all = torch.from_numpy(synth.chunk(max(ms), 16)[0].view(np.int16)).cuda().view(torch.float16)
     w_all = torch.from_numpy(synth.chunk(16, max(ns))[1].view(np.int16)).cuda().view(torch.float16)
+    cases, keep, flops = [], [], {}
     for N in ns:
         for M in ms:
             per = (M + N) * K * 2
@@ -703,51 +766,80 @@ def gemm_sweep(quick=False):
             As = [a_all[:M].clone() for _ in range(copies)]
             Ws = [w_all[:N].clone() for _ in range(copies)]
             C = torch.empty((M, N), dtype=torch.float16, device="cuda")
-            calls = [(lambda A=As[i], W=Ws[i]: mr.gemm_f16(A, W, C)) for i in range(copies)]
-            us = _time_calls(torch, calls)
-            tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
-            out["chunk"][f"{M}x{N}"] = {"us": us, "TFLOPs": tf,
-                                        "tile": mr.gemm_f16_tile_name(mr.gemm_f16_select_tile(M, N, K))}
-            del As, Ws, C
-    big = [v["TFLOPs"] for k, v in out["chunk"].items() if int(k.split("x")[0]) >= 1024]
+            keep.append((As, Ws, C))
+
+            def calls(As=As, Ws=Ws, C=C):
+                for A, W in zip(As, Ws):
+                    mr.gemm_f16(A, W, C)
+            cases.append((("chunk", f"{M}x{N}"), graph_of(torch, stream, calls), copies, 1))
+            flops[("chunk", f"{M}x{N}")] = 2.0 * M * N * K
     # narrow: one A per M shared by 36 different W[96, 2560]
     w96 = [torch.from_numpy(synth.narrow(1, w_index=i)[1].view(np.int16)).cuda().view(torch.float16)
            for i in range(36)]
     for M in (NARROW_M if not quick else (2048,)):
         a16 = torch.from_numpy(synth.narrow(M)[0].view(np.int16)).cuda().view(torch.float16)
         C = torch.empty((M, 96), dtype=torch.float16, device="cuda")
-        calls = [(lambda W=w96[i]: mr.gemm_f16(a16, W, C)) for i in range(36)]
-        us = _time_calls(torch, calls)
         Cs = [torch.empty((M, 96), dtype=torch.float16, device="cuda") for _ in range(36)]
-        ug = _time_calls(torch, [lambda: mr.gemm_f16_grouped(a16, w96, Cs)] * 4)
-        out["narrow"][str(M)] = {"us_per_call": us, "us_per_36_calls": 36 * us,
-                                 "TFLOPs": 2.0 * M * 96 * K / (us * 1e-6) / 1e12,
-                                 "tile": mr.gemm_f16_tile_name(mr.gemm_f16_select_tile(M, 96, K)),
-                                 "grouped_us_for_36": ug,
-                                 "grouped_TFLOPs": 36 * 2.0 * M * 96 * K / (ug * 1e-6) / 1e12,
-                                 "grouped_tile": mr.gemm_f16_tile_name(
-                                     mr.gemm_f16_grouped_select_tile(M, 96, K, 36))}
+        keep.append((a16, C, Cs))
+
+        def singles(a16=a16, C=C):
+            for W in w96:
+                mr.gemm_f16(a16, W, C)
+
+        def grouped(a16=a16, Cs=Cs):
+            for _ in range(4):
+                mr.gemm_f16_grouped(a16, w96, Cs)
+        cases.append((("narrow", M), graph_of(torch, stream, singles), 36, 1))
+        cases.append((("narrow_grouped", M), graph_of(torch, stream, grouped), 4, 1))
     # Tile-order study (the analogue of the audit's SLC swizzle): same bits,
-    # timed for several column-band widths.
-    study = {}
+    # timed for several column-band widths (operands warm in L2).
+    same_bits = {}
     for (M, N) in ((2048, 6144), (1983, 4096), (448, 6144)):
-        A = a_all[:M]
-        W = w_all[:N]
+        A, W = a_all[:M], w_all[:N]
         ref = None
-        row = {}
         for raster in (0, 2, 4, 8):
             C = torch.empty((M, N), dtype=torch.float16, device="cuda")
-            us = _time_calls(torch, [lambda C=C, r=raster: mr.gemm_f16(A, W, C, raster=r)] * 8)
-            torch.cuda.synchronize()
-            same = True if ref is None else bool(torch.equal(C.view(torch.int16), ref.view(torch.int16)))
+            keep.append(C)
+
+            def calls(A=A, W=W, C=C, r=raster):
+                for _ in range(8):
+                    mr.gemm_f16(A, W, C, raster=r)
+            cases.append((("raster", f"{M}x{N}", raster), graph_of(torch, stream, calls), 8, 1))
+            same_bits[(f"{M}x{N}", raster)] = True if ref is None else bool(
+                torch.equal(C.view(torch.int16), ref.view(torch.int16)))
             ref = C if ref is None else ref
-            row[str(raster)] = {"us": us, "TFLOPs": 2.0 * M * N * K / (us * 1e-6) / 1e12, "same_bits": same}
-        study[f"{M}x{N}"] = row
-    out["raster_study"] = study
+    t = interleaved(torch, stream, cases)
+    out = {"chunk": {}, "narrow": {}, "raster_study": {}}
+    for N in ns:
+        for M in ms:
+            key = ("chunk", f"{M}x{N}")
+            out["chunk"][f"{M}x{N}"] = {"us": t[key]["min"], "us_median": t[key]["median"],
+                                        "TFLOPs": flops[key] / (t[key]["min"] * 1e-6) / 1e12,
+                                        "tile": mr.gemm_f16_tile_name(mr.gemm_f16_select_tile(M, N, K))}
+    for M in (NARROW_M if not quick else (2048,)):
+        us, ug = t[("narrow", M)]["min"], t[("narrow_grouped", M)]["min"]
+        out["narrow"][str(M)] = {"us_per_call": us, "us_per_call_median": t[("narrow", M)]["median"],
+                                 "us_per_36_calls": 36 * us, "TFLOPs": 2.0 * M * 96 * K / (us * 1e-6) / 1e12,
+                                 "tile": mr.gemm_f16_tile_name(mr.gemm_f16_select_tile(M, 96, K)),
+                                 "grouped_us_for_36": ug, "grouped_us_for_36_median": t[("narrow_grouped", M)]["median"],
+                                 "grouped_TFLOPs": 36 * 2.0 * M * 96 * K / (ug * 1e-6) / 1e12,
+                                 "grouped_tile": mr.gemm_f16_tile_name(mr.gemm_f16_grouped_select_tile(M, 96, K, 36))}
+    for (M, N) in ((2048, 6144), (1983, 4096), (448, 6144)):
+        out["raster_study"][f"{M}x{N}"] = {
+            str(r): {"us": t[("raster", f"{M}x{N}", r)]["min"],
+                     "TFLOPs": 2.0 * M * N * K / (t[("raster", f"{M}x{N}", r)]["min"] * 1e-6) / 1e12,
+                     "same_bits": same_bits[(f"{M}x{N}", r)]} for r in (0, 2, 4, 8)}
+    big = [v["TFLOPs"] for k, v in out["chunk"].items() if int(k.split("x")[0]) >= 1024]
+    big_n = [v["TFLOPs"] for k, v in out["chunk"].items()
+             if int(k.split("x")[0]) >= 1024 and int(k.split("x")[1]) >= 4096]
     out["summary"] = {"tflops_M_ge_1024_mean": float(np.mean(big)) if big else None,
                       "tflops_M_ge_1024_max": float(np.max(big)) if big else None,
-                      "peak_bf16_tflops": tf_burst, "peak_kind": kind,
-                      "frac_of_peak_mean": (float(np.mean(big)) / tf_burst) if big else None}
+                      "tflops_M_ge_1024_N_ge_4096_mean": float(np.mean(big_n)) if big_n else None,
+                      "peak_bf16_tflops": tf_burst, "peak_bf16_tflops_sustained": tf_sus, "peak_kind": kind,
+                      "frac_of_peak_mean": (float(np.mean(big)) / tf_burst) if big else None,
+                      "method": f"min (and median) over {ROUNDS} interleaved rounds; operands rotated over "
+                                "copies > 2x L2 (raster study: warm)"}
+    del cases, keep
     return out
 
 
@@ -797,14 +889,16 @@ def path_sweep():
     (k=2560, n=6144) weights: us_per_row of the multi-row GEMV (m > 16 runs as
     16-row groups, each re-reading the weight) and of the tcgen05 GEMM (bf16
     in, fp32 out, auto tile), and the smallest m at which the GEMM is faster.
-    Weights rotate over copies larger than 2x L2."""
+    Weights rotate over copies larger than 2x L2; min and median over
+    interleaved rounds."""
     import numpy as np
     import torch
     import synth
     import verify_weight_streaming_b200 as mr
     props = torch.cuda.get_device_properties(0)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
-    res = {}
+    stream = torch.cuda.Stream()
+    cases, keep = [], []
     for name, k, n, wl in (("k896_n4864", 896, 4864, synth.WL_GEMV_FFN),
                            ("k2560_n6144", 2560, 6144, synth.WL_SWEEP)):
         a16 = synth.normal_bits(synth.seed_for(wl, 0), (max(SWEEP_M), k), "bf16", 1.0)
@@ -815,30 +909,39 @@ def path_sweep():
         Ws = [w.clone() for _ in range(copies)]
         Ab = A.view(torch.bfloat16)
         Wb = [x.view(torch.bfloat16) for x in Ws]
-        curve = {}
-        cross = None
+        keep.append((A, Ws))
         for m in SWEEP_M:
             C = torch.empty((m, n), dtype=torch.float32, device="cuda")
+            keep.append(C)
             groups = [(r0, min(16, m - r0)) for r0 in range(0, m, 16)]
-            calls = []
-            for i in range(copies):
-                def gemv_call(i=i):
+
+            def gemv_calls(C=C, groups=groups):
+                for W in Ws:
                     for r0, rr in groups:
-                        mr.mrgemv_bf16(A[r0:r0 + rr], Ws[i], C[r0:r0 + rr], flags=mr.MR_GEMV_PDL)
-                calls.append(gemv_call)
-            t_gemv = _time_calls(torch, calls, reps=2)
-            gcalls = [(lambda i=i: mr.gemm_f16(Ab[:m], Wb[i], C)) for i in range(copies)]
-            t_gemm = _time_calls(torch, gcalls, reps=2)
+                        mr.mrgemv_bf16(A[r0:r0 + rr], W, C[r0:r0 + rr], flags=mr.MR_GEMV_PDL)
+
+            def gemm_calls(C=C, m=m):
+                for W in Wb:
+                    mr.gemm_f16(Ab[:m], W, C)
+            cases.append(((name, m, "gemv"), graph_of(torch, stream, gemv_calls), copies, 1))
+            cases.append(((name, m, "gemm"), graph_of(torch, stream, gemm_calls), copies, 1))
+    t = interleaved(torch, stream, cases)
+    res = {}
+    for name, k, n in (("k896_n4864", 896, 4864), ("k2560_n6144", 2560, 6144)):
+        curve, cross = {}, None
+        for m in SWEEP_M:
+            t_gemv, t_gemm = t[(name, m, "gemv")]["min"], t[(name, m, "gemm")]["min"]
             curve[str(m)] = {"gemv_us_per_row": t_gemv / m, "gemm_us_per_row": t_gemm / m,
                              "gemv_us": t_gemv, "gemm_us": t_gemm,
+                             "gemv_us_median": t[(name, m, "gemv")]["median"],
+                             "gemm_us_median": t[(name, m, "gemm")]["median"],
                              "gemm_TFLOPs": 2.0 * m * n * k / (t_gemm * 1e-6) / 1e12,
                              "gemm_tile": mr.gemm_f16_tile_name(mr.gemm_f16_select_tile(m, n, k))}
             if cross is None and t_gemm <= t_gemv:
                 cross = m
-            del C
         res[name] = {"curve": curve, "crossover_m": cross,
                      "note": "GEMV for m > 16 is ceil(m/16) calls of up to 16 rows; GEMM is one call"}
-        del Ws, Wb, w
+    del cases, keep
     return res
 
 

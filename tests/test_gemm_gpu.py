@@ -214,3 +214,32 @@ def test_raster_orders_give_identical_bits(M, N, tile):
             ref = raw
             check(synth.bits_to_float32(raw.view(np.uint16), "f16")[:64], a[:64], w, "f16", "f16")
         assert np.array_equal(raw, ref), raster
+
+
+# ------------------------------------------------------ full-size parity
+# Every element of the output against the fp64 oracle, at the full prompt-chunk
+# sizes (the oracle takes tens of seconds on the host's cores for each).
+
+def test_full_parity_1983x1152_f16():
+    """The Wk chunk shape (M % 128 = 63, a tail tile), f16 in and out, auto tile."""
+    a, w = synth.chunk(1983, 1152)
+    c, _ = run_gemm(a, w)
+    check(c, a, w, "f16", "f16")
+
+
+def test_full_parity_1024x6144_bf16_to_f32():
+    """The m-sweep's GEMM path: bf16 in, fp32 out, K = 2560, N = 6144."""
+    a = synth.normal_bits(synth.seed_for(synth.WL_SWEEP, 0), (1024, 2560), "bf16", 1.0)
+    w = synth.normal_bits(synth.seed_for(synth.WL_SWEEP, 1), (6144, 2560), "bf16", 1.0 / np.sqrt(2560))
+    c, _ = run_gemm(a, w, in_fmt="bf16", out_fmt="f32")
+    check(c, a, w, "bf16", "f32")
+
+
+def test_full_parity_grouped_36_narrow_at_2048():
+    """All 36 N = 96 outputs of one grouped launch at M = 2048, every element
+    (the oracle runs once on the 36 weights stacked: the same per-element sum)."""
+    a = synth.narrow(2048)[0]
+    ws = [synth.narrow(1, w_index=i)[1] for i in range(36)]
+    outs = run_grouped(a, ws)
+    c = np.concatenate([synth.bits_to_float32(o.view(np.uint16), "f16") for o in outs], axis=1)
+    check(c, a, np.concatenate(ws, axis=0), "f16", "f16")

@@ -9,6 +9,10 @@
 
 #include "mrgemm.h"
 
+#ifndef MR_WAIT_TEST_FIRST
+#define MR_WAIT_TEST_FIRST 1
+#endif
+
 namespace mr {
 
 // Per-device error word: bits MR_DEVERR_*, set by a kernel whose bounded wait
@@ -67,10 +71,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of phase `parity` (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for phase `parity` of the barrier to complete, for at most limit_ns.
 // Returns false (after recording `err_bits`) when the limit runs out.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t err_bits,
                                                   uint64_t limit_ns = kWaitLimitNs) {
+#if MR_WAIT_TEST_FIRST
+    if (mbar_test_wait(bar, parity)) return true;
+#endif
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
         if (mbar_try_wait(bar, parity)) return true;

@@ -14,15 +14,18 @@
 //    counted on an mbarrier (no tensor map; each copy lands in its own CTA).
 //    Group g is consumed by column warp g % CWG from slot g % S; when slots
 //    are refilled, S is a multiple of CWG, so each slot has a single consumer
-//    warp that waits for the slot's successive uses in order.  The first slots
-//    are requested before griddepcontrol.wait, so under programmatic
-//    dependent launch the weight stream overlaps the previous kernel.
-//  * KW x CWG warps per CTA, at most 16 (8 for the 8-row, 8-column kernel).
-//    More warps than k-slices work on separate column groups in parallel.
+//    warp that waits for the slot's successive uses in order.  The whole first
+//    pass of the ring is requested before griddepcontrol.wait, so under
+//    programmatic dependent launch the weight streams while the previous
+//    kernel runs.
+//  * KW x CWG warps per CTA, at most 16.  More warps than k-slices work on
+//    separate column groups in parallel.
 //  * A (m rows, bf16) is staged once in shared memory by a bulk copy issued
-//    after the grid-dependency wait, right after the first weight chunk and
-//    before the others (copies from one CTA are served roughly in order, so A
-//    must not queue behind the whole weight block); rows m..MB-1 are zero.
+//    after the grid-dependency wait; rows m..MB-1 are zero.
+//  * The k loop reads shared memory with loads the compiler may schedule
+//    freely (their addresses pass through a volatile move after the slot's
+//    barrier wait, and every accumulator is pinned before the slot is
+//    released), and advances two rows' chains per fma.rn.f32x2.
 //  * Lanes split k in 4-element chunks: chunk q belongs to lane q % 32 of the
 //    k-slice that holds it.  KW warps split k into contiguous slices; KW is a
 //    function of k alone.  Each lane keeps one fp32 accumulator per (row,
@@ -45,15 +48,19 @@
 namespace mr {
 namespace gemv {
 
-// Warps per CTA at most, and the unroll of the k loop, per (rows, columns per
-// group).  16 warps (512 threads, so at most 128 registers each) give the
-// FMA-bound shapes twice the warps to hide shared-memory and FMA latency; the
-// 8-row, 8-column kernel needs ~230 registers for its accumulators and W
-// operands and keeps 8 warps.  The 8- and 16-row kernels fit 128 registers
-// only without unrolling the k loop.  None of this changes an output's
-// arithmetic: a lane's chain and the reduction order are fixed by k.
-__host__ __device__ constexpr int warps_max(int MB, int CG) { return (MB == 8 && CG == 8) ? 8 : 16; }
-__host__ __device__ constexpr int q_unroll(int MB, int CG) { return (MB >= 8 && warps_max(MB, CG) == 16) ? 1 : 2; }
+// Warps per CTA at most (512 threads, so at most 128 registers each: a CTA
+// of fewer warps then leaves room on its SM for the next launch's CTA), and
+// the unroll of the k loop.  None of this changes an output's arithmetic: a
+// lane's chain and the reduction order are fixed by k.
+#ifndef MR_GEMV_UNROLL_SMALL
+#define MR_GEMV_UNROLL_SMALL 2
+#endif
+#ifndef MR_GEMV_UNROLL_LARGE
+#define MR_GEMV_UNROLL_LARGE 1
+#endif
+constexpr int kWarpsMax = 16;
+__host__ __device__ constexpr int warps_max(int, int) { return kWarpsMax; }
+__host__ __device__ constexpr int q_unroll(int MB, int) { return MB >= 8 ? MR_GEMV_UNROLL_LARGE : MR_GEMV_UNROLL_SMALL; }
 constexpr int kMaxRows = 16;
 
 struct Params {
@@ -81,11 +88,24 @@ struct Params {
 
 // k-slice split: a function of k alone (never of m), so the reduction tree of
 // an output element is fixed by k.
+#ifndef MR_GEMV_MIN_CHUNKS
+#define MR_GEMV_MIN_CHUNKS 4   // 4-element chunks per lane per k-slice, at least
+#endif
+#ifndef MR_GEMV_EVEN_LANES
+#define MR_GEMV_EVEN_LANES 1   // every lane of a slice gets the same number of chunks
+#endif
+#ifndef MR_GEMV_KW_MAX
+#define MR_GEMV_KW_MAX 4
+#endif
 __host__ __device__ inline int k_warps(int k) {
     const int q = k / 4;
-    if (q % 128 == 0 && q >= 512) return 4;
-    if (q % 64 == 0 && q >= 256) return 2;
-    return 1;
+    int best = 1;
+    for (int kw = 2; kw <= MR_GEMV_KW_MAX; kw *= 2) {
+        if (q % kw != 0 || q / kw < 32 * MR_GEMV_MIN_CHUNKS) break;
+        if (MR_GEMV_EVEN_LANES && (q / kw) % 32 != 0) break;
+        best = kw;
+    }
+    return best;
 }
 
 // The shared expert's scalar gate: logistic of the GEMV output, with CUDA's
@@ -98,28 +118,27 @@ __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w <
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // 8-byte load from shared memory by 32-bit shared address (always LDS, never
-// a generic load).
+// a generic load).  Not volatile: the compiler may schedule it like any
+// load, so its address must come from launder() after the wait that makes
+// the data valid (that dependence keeps it below the wait).
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
     uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
     return v;
 }
 
-// Packed pairs of fp32 in one 64-bit register pair (low half first).
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void unpack2(uint64_t v, float &lo, float &hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+// The same value, through an instruction the compiler cannot see through or
+// move across other volatile asm (the barrier waits): loads whose addresses
+// derive from it stay after the wait that precedes it.
+__device__ __forceinline__ uint32_t launder(uint32_t x) {
+    uint32_t y;
+    asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x) : "memory");
+    return y;
 }
 
-// acc.lo = fma(a.lo, b.lo, acc.lo); acc.hi = fma(a.hi, b.hi, acc.hi): two
-// independent round-to-nearest fp32 FMAs in one instruction.
-__device__ __forceinline__ void ffma2(uint64_t &acc, uint64_t a, uint64_t b) {
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
-}
+// acc.x = fma(a.x, b.x, acc.x); acc.y = fma(a.y, b.y, acc.y): two independent
+// round-to-nearest fp32 FMAs in one instruction (fma.rn.f32x2).
+__device__ __forceinline__ void ffma2(float2 &acc, float2 a, float2 b) { acc = __ffma2_rn(a, b, acc); }
 
 // Reduce-scatter over the warp: level D pairs lanes that differ in bit D (16,
 // 8, 4, 2, 1 in that order).  While more than one value is left, the lane with
@@ -172,7 +191,7 @@ struct Smem {
     uint64_t *chunk_full; // [S] first pass: one barrier per up-front copy chunk
     uint64_t *full;       // [S] refills: slot s's uses 1, 2, ...
     uint64_t *empty;      // [S]
-    uint64_t *a_full;     // [1] A has landed
+    uint64_t *a_full;     // [1] A has landed (A staged by a bulk copy)
     uint64_t *parts_done; // [1] every warp has written its k-slice partials
     uint64_t *cta_done;   // [1] every warp's logits are stored (fused router)
     uint64_t *decided;    // [1] thread 0 knows whether this CTA finished last
@@ -195,47 +214,86 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     const uint32_t par = g < p.S ? 0u : (uint32_t)(g / p.S - 1) & 1u;
     if (!mbar_wait_bounded(smem_u32(bar), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
 
-    const uint32_t w_s = smem_u32(sm.ring + (size_t)slot * p.slot_bytes);
-    const uint32_t a_s = smem_u32(sm.a);
+    const uint32_t w_s = launder(smem_u32(sm.ring + (size_t)slot * p.slot_bytes));
+    const uint32_t a_s = launder(smem_u32(sm.a));
     const uint32_t row_b = (uint32_t)k * 2u;
     // acc[rp][j] holds rows (2rp, 2rp+1) of column j: one fp32 chain per
     // (row, column), over this lane's k positions in ascending order.
     constexpr int RP = MB / 2;
-    uint64_t acc[RP][NC];
+    float2 acc[RP][NC];
 #pragma unroll
     for (int rp = 0; rp < RP; ++rp)
 #pragma unroll
-        for (int j = 0; j < NC; ++j) acc[rp][j] = 0ull;
+        for (int j = 0; j < NC; ++j) acc[rp][j] = make_float2(0.0f, 0.0f);
 
+    // The loads are software-pipelined by hand: the next row pair's A (or the
+    // next column's W, or the next chunk's first operands) is requested
+    // before the current FMAs issue, so one warp per scheduler does not wait
+    // out each shared-memory load.  The FMA sequence of every chain is the
+    // same as without pipelining.
+    auto a_at = [&](int r, int qq) { return lds64(a_s + (uint32_t)r * row_b + 8u * (uint32_t)qq); };
+    auto w_at = [&](int j, int qq) { return lds64(w_s + (uint32_t)j * row_b + 8u * (uint32_t)qq); };
 #pragma unroll (q_unroll(MB, CGMAX))
     for (int q = q_begin + lane; q < q_end; q += 32) {
-        uint64_t wd[4][NC];  // (w, w) for element e of the chunk, column j
+        if constexpr (RP < NC) {
+            float2 ap[RP][4];
 #pragma unroll
-        for (int j = 0; j < NC; ++j) {
-            const uint2 raw = lds64(w_s + (uint32_t)j * row_b + 8u * (uint32_t)q);
-            const float w0 = bf16lo(raw.x), w1 = bf16hi(raw.x), w2 = bf16lo(raw.y), w3 = bf16hi(raw.y);
-            wd[0][j] = pack2(w0, w0);
-            wd[1][j] = pack2(w1, w1);
-            wd[2][j] = pack2(w2, w2);
-            wd[3][j] = pack2(w3, w3);
-        }
-#pragma unroll
-        for (int rp = 0; rp < RP; ++rp) {
-            const uint2 r0 = lds64(a_s + (uint32_t)(2 * rp) * row_b + 8u * (uint32_t)q);
-            const uint2 r1 = lds64(a_s + (uint32_t)(2 * rp + 1) * row_b + 8u * (uint32_t)q);
-            const uint64_t a0 = pack2(bf16lo(r0.x), bf16lo(r1.x));
-            const uint64_t a1 = pack2(bf16hi(r0.x), bf16hi(r1.x));
-            const uint64_t a2 = pack2(bf16lo(r0.y), bf16lo(r1.y));
-            const uint64_t a3 = pack2(bf16hi(r0.y), bf16hi(r1.y));
+            for (int rp = 0; rp < RP; ++rp) {
+                const uint2 r0 = a_at(2 * rp, q), r1 = a_at(2 * rp + 1, q);
+                ap[rp][0] = make_float2(bf16lo(r0.x), bf16lo(r1.x));
+                ap[rp][1] = make_float2(bf16hi(r0.x), bf16hi(r1.x));
+                ap[rp][2] = make_float2(bf16lo(r0.y), bf16lo(r1.y));
+                ap[rp][3] = make_float2(bf16hi(r0.y), bf16hi(r1.y));
+            }
 #pragma unroll
             for (int j = 0; j < NC; ++j) {
-                ffma2(acc[rp][j], a0, wd[0][j]);
-                ffma2(acc[rp][j], a1, wd[1][j]);
-                ffma2(acc[rp][j], a2, wd[2][j]);
-                ffma2(acc[rp][j], a3, wd[3][j]);
+                const uint2 raw = w_at(j, q);
+                const float w0 = bf16lo(raw.x), w1 = bf16hi(raw.x), w2 = bf16lo(raw.y), w3 = bf16hi(raw.y);
+                const float2 d0 = make_float2(w0, w0), d1 = make_float2(w1, w1), d2 = make_float2(w2, w2),
+                             d3 = make_float2(w3, w3);
+#pragma unroll
+                for (int rp = 0; rp < RP; ++rp) {
+                    ffma2(acc[rp][j], ap[rp][0], d0);
+                    ffma2(acc[rp][j], ap[rp][1], d1);
+                    ffma2(acc[rp][j], ap[rp][2], d2);
+                    ffma2(acc[rp][j], ap[rp][3], d3);
+                }
+            }
+        } else {
+            float2 wd[4][NC];
+#pragma unroll
+            for (int j = 0; j < NC; ++j) {
+                const uint2 raw = w_at(j, q);
+                const float w0 = bf16lo(raw.x), w1 = bf16hi(raw.x), w2 = bf16lo(raw.y), w3 = bf16hi(raw.y);
+                wd[0][j] = make_float2(w0, w0);
+                wd[1][j] = make_float2(w1, w1);
+                wd[2][j] = make_float2(w2, w2);
+                wd[3][j] = make_float2(w3, w3);
+            }
+#pragma unroll
+            for (int rp = 0; rp < RP; ++rp) {
+                const uint2 r0 = a_at(2 * rp, q), r1 = a_at(2 * rp + 1, q);
+                const float2 a0 = make_float2(bf16lo(r0.x), bf16lo(r1.x));
+                const float2 a1 = make_float2(bf16hi(r0.x), bf16hi(r1.x));
+                const float2 a2 = make_float2(bf16lo(r0.y), bf16lo(r1.y));
+                const float2 a3 = make_float2(bf16hi(r0.y), bf16hi(r1.y));
+#pragma unroll
+                for (int j = 0; j < NC; ++j) {
+                    ffma2(acc[rp][j], a0, wd[0][j]);
+                    ffma2(acc[rp][j], a1, wd[1][j]);
+                    ffma2(acc[rp][j], a2, wd[2][j]);
+                    ffma2(acc[rp][j], a3, wd[3][j]);
+                }
             }
         }
     }
+    // Every accumulator is final before the slot is released: the empty
+    // volatile asm consumes them all, and volatile asm keeps its order, so no
+    // load of the slot (nor the FMAs that use it) can sink below the release.
+#pragma unroll
+    for (int rp = 0; rp < RP; ++rp)
+#pragma unroll
+        for (int j = 0; j < NC; ++j) asm volatile("" ::"f"(acc[rp][j].x), "f"(acc[rp][j].y));
     // This warp no longer reads the slot.
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&sm.empty[slot]));
@@ -246,7 +304,8 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     for (int rp = 0; rp < RP; ++rp)
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
-            unpack2(acc[rp][j], v[(2 * rp) * NC + j], v[(2 * rp + 1) * NC + j]);
+            v[(2 * rp) * NC + j] = acc[rp][j].x;
+            v[(2 * rp + 1) * NC + j] = acc[rp][j].y;
         }
     int base = 0;
     ReduceScatter<V, 16>::run(v, lane, base);
@@ -286,7 +345,7 @@ __device__ __forceinline__ bool run_group(const Params &p, const Smem &sm, int g
 }
 
 template <int MB, int CG, bool FUSED>
-__global__ void __launch_bounds__(warps_max(MB, CG) * 32, 1) gemv_kernel(const Params p) {
+__global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
 
     const int tid = threadIdx.x;
@@ -306,13 +365,14 @@ __global__ void __launch_bounds__(warps_max(MB, CG) * 32, 1) gemv_kernel(const P
     sm.chunk_full = reinterpret_cast<uint64_t *>(sm.ring + (size_t)p.S * p.slot_bytes);
     sm.full = sm.chunk_full + p.S;
     sm.empty = sm.full + p.S;
-    sm.a_full = sm.empty + p.S;
-    sm.cta_done = sm.a_full + 1;
-    sm.decided = sm.a_full + 2;
-    sm.is_last = reinterpret_cast<uint32_t *>(sm.a_full + 3);
-    sm.staged = sm.a_full + 4;
-    sm.parts_done = sm.a_full + 5;
-    sm.red = reinterpret_cast<float *>(sm.a_full + 6);
+    uint64_t *misc = sm.empty + p.S;  // 6 words: barriers and the last-CTA flag
+    sm.a_full = misc;
+    sm.cta_done = misc + 1;
+    sm.decided = misc + 2;
+    sm.is_last = reinterpret_cast<uint32_t *>(misc + 3);
+    sm.staged = misc + 4;
+    sm.parts_done = misc + 5;
+    sm.red = reinterpret_cast<float *>(misc + 6);
 
     // Groups per copy chunk when no slot is refilled (0 when slots are refilled).
     const int chunk_groups = (int)max(1u, (32768u + p.slot_bytes - 1) / p.slot_bytes);
@@ -365,11 +425,12 @@ __global__ void __launch_bounds__(warps_max(MB, CG) * 32, 1) gemv_kernel(const P
             mbar_init(smem_u32(sm.staged), 1);
         }
         fence_mbar_init();
-        // The first min(ng, S) groups come in chunks of whole groups of
-        // >= 32 KB each (small bulk copies stream below HBM bandwidth: ~2.6
-        // TB/s for 4 KB copies, ~6.2 TB/s for 16 KB, ~7 TB/s for 32-64 KB).
-        // Chunk 0 is requested now, before the wait for the previous kernel.
-        issue_chunk(0);
+        // The whole first pass of the ring (min(ng, S) groups) is requested
+        // now, before the wait for the previous kernel, in chunks of whole
+        // groups of >= 32 KB each (small bulk copies stream below HBM
+        // bandwidth: ~2.6 TB/s for 4 KB copies, ~6.2 TB/s for 16 KB, ~7 TB/s
+        // for 32-64 KB).  The weight does not depend on the previous kernel.
+        for (int c = 0; c * chunk_groups < first; ++c) issue_chunk(c);
     }
     // The weight stream is in flight; the next kernel may start launching.
     grid_launch_dependents();
@@ -377,9 +438,10 @@ __global__ void __launch_bounds__(warps_max(MB, CG) * 32, 1) gemv_kernel(const P
     grid_dependency_wait();
 
     // Stage A (bf16) in shared memory with one bulk copy (per row if strided);
-    // rows m..MB-1 are zero.  Only the first weight chunk was requested
-    // before this point, so A does not queue behind the whole weight stream;
-    // the remaining chunks follow it.
+    // rows m..MB-1 are zero.  Under programmatic dependent launch the weight
+    // was requested while the previous kernel ran and has mostly landed by
+    // now.  (Per-thread cp.async copies of A measured slower: up to 3 us for
+    // 16 rows of 2560, since every CTA reads the same A lines.)
     if (tid == 0) {
         const uint32_t row_bytes = (uint32_t)k * 2u;
         const uint32_t bar = smem_u32(sm.a_full);
@@ -390,7 +452,6 @@ __global__ void __launch_bounds__(warps_max(MB, CG) * 32, 1) gemv_kernel(const P
             for (int r = 0; r < p.m; ++r)
                 bulk_g2s(smem_u32(sm.a + (size_t)r * k), p.A + (int64_t)r * p.lda, row_bytes, bar);
         }
-        for (int c = 1; c * chunk_groups < first; ++c) issue_chunk(c);
     }
     {
         const int chunks = k / 8;  // 16-byte chunks per row
@@ -530,7 +591,10 @@ using KernelFn = void (*)(const Params);
 // accumulators per lane (MB x CG), and slots of about 20 KB for long rows, so
 // that a CTA's whole weight block can be in flight at once (8 columns of a
 // 2560-element row would make 40 KB slots and force slot refills).
-inline int col_group_rt(int MB, int k) { return (MB <= 8 && k <= 1536) ? 8 : 4; }
+#ifndef MR_GEMV_CG8_MAX_K
+#define MR_GEMV_CG8_MAX_K 1536
+#endif
+inline int col_group_rt(int MB, int k) { return (MB <= 8 && k <= MR_GEMV_CG8_MAX_K) ? 8 : 4; }
 
 template <bool FUSED>
 KernelFn kernel_for_mb(int MB, int CG) {
@@ -601,7 +665,10 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     const size_t red_bytes = red_floats(pl.KW, ng_max, pl.MB, pl.CG) * sizeof(float);
     const size_t topk_bytes = fused ? (size_t)warps_max(pl.MB, pl.CG) * 64 * 8 : 0;
     const size_t fixed = topk_bytes + pl.a_bytes + 24 * (size_t)ng_max + 48 + red_bytes + 64;
-    const size_t pdl_budget = 110 * 1024;
+#ifndef MR_GEMV_PDL_BUDGET_KB
+#define MR_GEMV_PDL_BUDGET_KB 110
+#endif
+    const size_t pdl_budget = MR_GEMV_PDL_BUDGET_KB * 1024;
     const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, (size_t)optin) : (size_t)optin;
     auto slots_for = [&](size_t b) -> int {
         if (b <= fixed) return 0;
