@@ -120,9 +120,10 @@ mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t flags, int3
  * router_gemv_topk -- the router in one launch: the multi-row GEMV of
  * mrgemv_bf16 followed by the per-row top-k of router_topk.  The two steps of
  * Strata PR #109 ("What", router bullet: one multi-row GEMV plus one multi-row
- * top-10 launch) are fused: the CTA that stores its logits last (an atomic
- * ticket in the workspace) selects the top-k of every row.  idx / val are
- * bitwise the outputs of mrgemv_bf16 then router_topk on the same inputs.
+ * top-10 launch) are fused: every CTA takes an atomic ticket in the workspace
+ * once its logits are stored, the last one advances a generation word there,
+ * and CTA r (one warp per row) then selects the top-k of row r.  idx / val
+ * are bitwise the outputs of mrgemv_bf16 then router_topk on the same inputs.
  *
  * A, Wt, m, n, k, lda, ldw, flags : as mrgemv_bf16_ex.
  * logits : NULL, or m rows of n fp32 (row stride ldl >= n) that receive the
@@ -131,7 +132,8 @@ mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t flags, int3
  * workspace : device memory, 256-byte aligned, of at least
  *          router_gemv_topk_workspace_bytes(m, n, logits != NULL) bytes.
  *          Its first MR_ROUTER_TICKET_BYTES must be zero before the first
- *          call; every completed call leaves them zero again.  Calls that may
+ *          call; every completed call leaves the ticket counter zero again
+ *          (and advances the generation word beside it).  Calls that may
  *          run at the same time (other streams) need separate workspaces.
  */
 #define MR_ROUTER_TICKET_BYTES 256u

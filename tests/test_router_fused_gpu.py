@@ -49,6 +49,7 @@ def test_fused_matches_two_launches(m, with_logits):
     if with_logits:
         assert np.array_equal(host(logits).view(np.uint32), c_ref.view(np.uint32))
     assert int(host(ws)[0]) == 0, "ticket not returned to zero"
+    assert int(host(ws)[16]) == 1, "one call advances the generation word once"
     ri, _ = oracle.topk(c_ref, 10)
     assert np.array_equal(host(idx), ri)
 

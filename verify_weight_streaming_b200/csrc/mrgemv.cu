@@ -62,6 +62,9 @@ constexpr int kWarpsMax = 16;
 __host__ __device__ constexpr int warps_max(int, int) { return kWarpsMax; }
 __host__ __device__ constexpr int q_unroll(int MB, int) { return MB >= 8 ? MR_GEMV_UNROLL_LARGE : MR_GEMV_UNROLL_SMALL; }
 constexpr int kMaxRows = 16;
+// Word of the fused router's ticket block that counts completed calls (the
+// counter itself is word 0; 64 bytes apart).
+constexpr int kGenerationWord = 16;
 
 struct Params {
     const uint16_t *A;
@@ -194,9 +197,7 @@ struct Smem {
     uint64_t *a_full;     // [1] A has landed (A staged by a bulk copy)
     uint64_t *parts_done; // [1] every warp has written its k-slice partials
     uint64_t *cta_done;   // [1] every warp's logits are stored (fused router)
-    uint64_t *decided;    // [1] thread 0 knows whether this CTA finished last
-    uint32_t *is_last;    // [2]
-    uint64_t *staged;     // [1] the last CTA's copy of the logits is complete
+    uint32_t *gen0;       // [2] the workspace's generation word before this call
     float *red;           // [groups][KW][MB x CG] k-slice partials (KW > 1)
 };
 
@@ -368,9 +369,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     uint64_t *misc = sm.empty + p.S;  // 6 words: barriers and the last-CTA flag
     sm.a_full = misc;
     sm.cta_done = misc + 1;
-    sm.decided = misc + 2;
-    sm.is_last = reinterpret_cast<uint32_t *>(misc + 3);
-    sm.staged = misc + 4;
+    sm.gen0 = reinterpret_cast<uint32_t *>(misc + 3);
     sm.parts_done = misc + 5;
     sm.red = reinterpret_cast<float *>(misc + 6);
 
@@ -419,11 +418,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
         }
         mbar_init(smem_u32(sm.a_full), 1);
         mbar_init(smem_u32(sm.parts_done), (uint32_t)(blockDim.x / 32));
-        if constexpr (FUSED) {
-            mbar_init(smem_u32(sm.cta_done), (uint32_t)(blockDim.x / 32));
-            mbar_init(smem_u32(sm.decided), 1);
-            mbar_init(smem_u32(sm.staged), 1);
-        }
+        if constexpr (FUSED) mbar_init(smem_u32(sm.cta_done), (uint32_t)(blockDim.x / 32));
         fence_mbar_init();
         // The whole first pass of the ring (min(ng, S) groups) is requested
         // now, before the wait for the previous kernel, in chunks of whole
@@ -436,6 +431,13 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     grid_launch_dependents();
     // A may be produced by the previous kernel on the stream.
     grid_dependency_wait();
+    if constexpr (FUSED) {
+        // The generation before this call: read after the previous kernel
+        // (possibly a fused call on the same workspace) has completed.
+        if (tid == 0)
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(*sm.gen0) : "l"(p.ticket + kGenerationWord)
+                         : "memory");
+    }
 
     // Stage A (bf16) in shared memory with one bulk copy (per row if strided);
     // rows m..MB-1 are zero.  Under programmatic dependent launch the weight
@@ -511,73 +513,55 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     }
 
     if constexpr (FUSED) {
-        // Router top-k in the same launch: the CTA that finishes its columns
-        // last (atomic ticket) selects the top-k of every row from the logits
-        // all CTAs stored.  Ordering: each warp's stores -> __syncwarp ->
-        // release arrive on cta_done (CTA scope) -> thread 0's acquire wait ->
-        // one acq_rel atomic at GPU scope, whose release covers what thread 0
-        // has observed; the last CTA's atomic acquires every other CTA's
-        // release, and hands it to its warps through the `decided` barrier.
-        // Every warp arrives even after a failed wait, so thread 0's wait ends.
+        // Router top-k in the same launch.  Every warp releases its logits
+        // (cta_done); thread 0 then takes a ticket (acq_rel at GPU scope).
+        // The CTA that draws the last ticket resets the counter and advances
+        // the workspace's generation word with a release store.  CTA b
+        // selects rows b, b + G, ... with one warp per row: lane 0 waits,
+        // bounded, for the generation to move past the value read after the
+        // grid-dependency wait, and the warp then reads the row from L2 (every
+        // CTA's stores are ordered before the last ticket, and that before
+        // the generation) and selects.  The m rows are selected in parallel
+        // on m SMs.  Every warp arrives even after a failed wait, so thread
+        // 0's wait ends.
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(sm.cta_done));
-        uint32_t last = 0;
-        if (warp == 0) {
-            // Warp 0 decides as a whole (its lanes never wait on different
-            // barriers); lane 0 takes the ticket.
-            if (mbar_wait_bounded(smem_u32(sm.cta_done), 0u, MR_DEVERR_GEMV_TIMEOUT)) {
-                if (lane == 0) {
-                    uint32_t t;
-                    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.ticket) : "memory");
-                    if (t == (uint32_t)p.G - 1u) {
-                        last = 1;
-                        *p.ticket = 0u;  // leave the counter at zero for the next call
-                    }
-                    *sm.is_last = last;
-                    mbar_arrive(smem_u32(sm.decided));
-                }
-            } else if (lane == 0) {
-                *sm.is_last = 0u;
-                mbar_arrive(smem_u32(sm.decided));
+        uint32_t *gen = p.ticket + kGenerationWord;
+        if (warp == 0 && mbar_wait_bounded(smem_u32(sm.cta_done), 0u, MR_DEVERR_GEMV_TIMEOUT) && lane == 0) {
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            uint32_t t;
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.ticket) : "memory");
+            if (t == (uint32_t)p.G - 1u) {
+                *p.ticket = 0u;  // the counter starts at zero for the next call
+                asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(gen), "r"(*sm.gen0 + 1u) : "memory");
             }
-            last = __shfl_sync(0xffffffffu, last, 0);
-        } else {
-            if (!mbar_wait_bounded(smem_u32(sm.decided), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
-            last = *sm.is_last;
         }
-        if (last == 0u) return;
-        // Stage every row's logits in shared memory (the A and ring regions are
-        // free now) with one bulk copy per row, all in flight together, when
-        // the rows are 16-byte aligned; otherwise read them from global memory.
         const int nwarps = blockDim.x >> 5;
-        const size_t region = p.a_bytes + (size_t)p.S * p.slot_bytes;
-        const uint32_t row_bytes = (uint32_t)p.n * 4u;
-        const bool staged = (size_t)p.m * row_bytes <= region && (row_bytes & 15u) == 0 &&
-                            ((uintptr_t)p.C & 15u) == 0 && (p.ldc & 3) == 0;
-        float *lg = reinterpret_cast<float *>(smem_raw);
-        if (staged) {
-            if (warp == 0) {
-                if (lane == 0) {
-                    // The logits were written by other CTAs through the generic
-                    // proxy; order them before the async-proxy reads.
-                    asm volatile("fence.proxy.async;" ::: "memory");
-                    const uint32_t bar = smem_u32(sm.staged);
-                    mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)p.m);
-                    for (int r = 0; r < p.m; ++r)
-                        bulk_g2s(smem_u32(lg + (size_t)r * p.n), p.C + (int64_t)r * p.ldc, row_bytes, bar);
+        int r = (int)blockIdx.x + warp * p.G;
+        if (r >= p.m) return;
+        uint32_t ok = 1u;
+        if (lane == 0) {
+            const uint32_t g0 = *sm.gen0;
+            const uint64_t t0 = globaltimer_ns();
+            uint32_t g;
+            for (int spin = 0;; ++spin) {
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(gen) : "memory");
+                if (g != g0) break;
+                if ((spin & 63) == 63 && globaltimer_ns() - t0 > kWaitLimitNs) {
+                    record_error(MR_DEVERR_GEMV_TIMEOUT);
+                    ok = 0u;
+                    break;
                 }
-                __syncwarp();
             }
-            if (!mbar_wait_bounded(smem_u32(sm.staged), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
         }
+        if (__shfl_sync(0xffffffffu, ok, 0) == 0u) return;
         uint64_t *tk = reinterpret_cast<uint64_t *>(sm.red + red_floats(p.KW, ng_max_of(p.n, p.G, CG), MB, CG)) + warp * 64;
-        for (int r = warp; r < p.m; r += nwarps) {
-            const float *x = staged ? lg + (size_t)r * p.n : p.C + (int64_t)r * p.ldc;
-            const uint64_t best = topk::warp_topk_fast<16>(x, p.n, p.topk, lane, 0, 1, 0ull, tk);
+        for (; r < p.m; r += nwarps * p.G) {
+            const float *x = p.C + (int64_t)r * p.ldc;
+            const uint64_t best = topk::warp_topk_fast<16, true>(x, p.n, p.topk, lane, 0, 1, 0ull, tk);
             if (lane < p.topk) {
-                const uint32_t j = topk::key_index(best);
-                p.idx[(int64_t)r * p.ldo + lane] = (int32_t)j;
-                if (p.val) p.val[(int64_t)r * p.ldo + lane] = topk::selected_value(best, x);
+                p.idx[(int64_t)r * p.ldo + lane] = (int32_t)topk::key_index(best);
+                if (p.val) p.val[(int64_t)r * p.ldo + lane] = topk::selected_value<true>(best, x);
             }
         }
     }

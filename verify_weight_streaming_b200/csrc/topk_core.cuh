@@ -38,12 +38,21 @@ __device__ __forceinline__ float key_value(uint64_t key, bool &exact) {
     return __uint_as_float(b);
 }
 
+// Row loads: plain, or (CG) cached in L2 only, for rows other CTAs of the
+// same grid have just written (an L1 line cached earlier could be stale).
+template <bool CG>
+__device__ __forceinline__ float load_row(const float *x, int j) {
+    if constexpr (CG) return __ldcg(x + j);
+    return x[j];
+}
+
 // Value to report for a selected key: decoded from the key when that is
 // exact, else re-read from the row.
+template <bool CG = false>
 __device__ __forceinline__ float selected_value(uint64_t key, const float *x) {
     bool exact;
     const float v = key_value(key, exact);
-    return exact ? v : x[key_index(key)];
+    return exact ? v : load_row<CG>(x, (int)key_index(key));
 }
 
 // Sort L keys descending (insertion network, compile-time indices).
@@ -176,7 +185,7 @@ __device__ __forceinline__ uint64_t warp_topk_merge(uint64_t (&key)[P], uint64_t
 
 // Running top-K of x[0, n) taken by one warp in chunks of 32*P elements
 // (chunks seg0, seg0 + seg_stride, ...), merged into `run`.
-template <int P>
+template <int P, bool CG = false>
 __device__ __forceinline__ uint64_t warp_topk_fast(const float *x, int n, int K, int lane, int seg0,
                                                    int seg_stride, uint64_t run, uint64_t *scratch) {
     for (int seg = seg0; (int64_t)seg * 32 * P < n; seg += seg_stride) {
@@ -185,7 +194,7 @@ __device__ __forceinline__ uint64_t warp_topk_fast(const float *x, int n, int K,
 #pragma unroll
         for (int i = 0; i < P; ++i) {
             const int j = base + lane + 32 * i;
-            v[i] = j < n ? x[j] : 0.0f;
+            v[i] = j < n ? load_row<CG>(x, j) : 0.0f;
         }
         uint64_t keys[P];
 #pragma unroll
