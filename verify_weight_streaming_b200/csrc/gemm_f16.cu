@@ -39,9 +39,9 @@
 namespace mr {
 namespace gemm {
 
-constexpr int BM = 128;          // rows per tile (MMA M)
 constexpr int BK = 64;           // K elements per k-block (128 bytes of 16-bit data)
-constexpr uint32_t kABytes = BM * BK * 2;
+constexpr int kMaxBM = 128;      // rows per tile (MMA M): 128, or 64 for tail-heavy M
+__host__ __device__ constexpr uint32_t a_bytes_for(int bm) { return (uint32_t)bm * BK * 2; }
 
 // Threads of a CTA: warps 0 and 6 producers (alternate ring stages), warp 1
 // MMA issue, warps 2-5 epilogue.
@@ -49,6 +49,7 @@ constexpr int kThreads = 224;
 constexpr int kProducers = 2;
 
 struct TileDesc {
+    int bm;         // rows per tile: 128, or 64 (tcgen05 M = 64: half of each lane quarter)
     int bn;
     int stages;     // k-block slots of shared memory
     int acc_cols;   // tensor-memory columns per accumulator buffer (power of two >= bn)
@@ -62,13 +63,14 @@ struct TileDesc {
 // The wider tiles keep one, since two 40-48 KB k-blocks per stage would leave
 // only two stages in flight.
 constexpr TileDesc kTiles[] = {
-    {32, 8, 32, 2, "128x32"},   {64, 8, 64, 2, "128x64"},   {96, 7, 128, 2, "128x96"},
-    {128, 6, 128, 2, "128x128"}, {192, 5, 256, 1, "128x192"}, {256, 4, 256, 1, "128x256"},
+    {128, 32, 8, 32, 2, "128x32"},   {128, 64, 8, 64, 2, "128x64"},   {128, 96, 7, 128, 2, "128x96"},
+    {128, 128, 6, 128, 2, "128x128"}, {128, 192, 5, 256, 1, "128x192"}, {128, 256, 4, 256, 1, "128x256"},
+    {64, 128, 8, 128, 2, "64x128"},   {64, 256, 5, 256, 1, "64x256"},
 };
 constexpr int kNumTiles = sizeof(kTiles) / sizeof(kTiles[0]);
 
-__host__ __device__ constexpr uint32_t smem_bytes_for(int bn, int stages) {
-    return (uint32_t)stages * (kABytes + (uint32_t)bn * BK * 2) + 1024 /*align*/ + 256 /*barriers*/;
+__host__ __device__ constexpr uint32_t smem_bytes_for(int bm, int bn, int stages) {
+    return (uint32_t)stages * (a_bytes_for(bm) + (uint32_t)bn * BK * 2) + 1024 /*align*/ + 256 /*barriers*/;
 }
 
 // ---- tcgen05 / TMA PTX wrappers --------------------------------------------
@@ -231,8 +233,9 @@ __device__ __forceinline__ void tile_coords(int t, int ntm, int ntn, int raster,
     nt = n0 + r % width;
 }
 
-template <int BN, int STAGES, int ACC_COLS, int KPB, int OUT, int MAXG>
+template <int BM, int BN, int STAGES, int ACC_COLS, int KPB, int OUT, int MAXG>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs<MAXG> args) {
+    constexpr uint32_t kABytes = a_bytes_for(BM);
     const CUtensorMap &tmA = args.tmA;
     const int M = args.M, N = args.N, K = args.K, G = args.G, P = args.P;
     const int64_t ldc = args.ldc;
@@ -390,7 +393,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const int m0 = mt * BM;
             const int g0 = P > 1 ? slot * P : slot / args.tn_per_group;
             const int n0 = P > 1 ? 0 : (slot % args.tn_per_group) * BN;
-            const int row = m0 + 32 * q + lane;
+            // M = 128: tensor-memory lane 32q + l holds row 32q + l of the tile.
+            // M = 64: lanes 32q .. 32q + 15 hold rows 16q .. 16q + 15 (the
+            // first half of each lane quarter); lanes 16..31 of the warp
+            // read unused lanes and store nothing.
+            const int row = BM == 128 ? m0 + 32 * q + lane : (lane < 16 ? m0 + 16 * q + lane : M);
             if (!mbar_wait_bounded(smem_u32(&acc_full[b]), (ti >> 1) & 1u, MR_DEVERR_GEMM_TIMEOUT)) break;
             tc_fence_after();
             const uint32_t acc = tmem + b * ACC_COLS + ((uint32_t)(32 * q) << 16);
@@ -427,7 +434,7 @@ using KernelFn = void (*)(const GemmArgs<MAXG>);
 
 template <int T, int OUT, int MAXG>
 constexpr KernelFn<MAXG> kernel_of() {
-    return gemm_kernel<kTiles[T].bn, kTiles[T].stages, kTiles[T].acc_cols, kTiles[T].kpb, OUT, MAXG>;
+    return gemm_kernel<kTiles[T].bm, kTiles[T].bn, kTiles[T].stages, kTiles[T].acc_cols, kTiles[T].kpb, OUT, MAXG>;
 }
 
 template <int OUT, int MAXG>
@@ -438,7 +445,9 @@ KernelFn<MAXG> pick_out(int t) {
         case 2: return kernel_of<2, OUT, MAXG>();
         case 3: return kernel_of<3, OUT, MAXG>();
         case 4: return kernel_of<4, OUT, MAXG>();
-        default: return kernel_of<5, OUT, MAXG>();
+        case 5: return kernel_of<5, OUT, MAXG>();
+        case 6: return kernel_of<6, OUT, MAXG>();
+        default: return kernel_of<7, OUT, MAXG>();
     }
 }
 
@@ -466,7 +475,7 @@ cudaError_t init_device(int device) {
     if (device >= 0 && device < 64 && !g_attr_done[device]) {
         for (int t = 0; t < kNumTiles; ++t)
             for (int out = 0; out < 3; ++out) {
-                const int smem = (int)smem_bytes_for(kTiles[t].bn, kTiles[t].stages);
+                const int smem = (int)smem_bytes_for(kTiles[t].bm, kTiles[t].bn, kTiles[t].stages);
                 cudaError_t e = cudaFuncSetAttribute(kernel_for<1>(t, out),
                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
                 if (e != cudaSuccess) return e;
@@ -496,9 +505,9 @@ bool encode_operand(CUtensorMap *map, const void *ptr, int64_t rows, int64_t col
 // Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), A and B
 // formats (bits 7-9, 10-12: 0 = f16, 1 = bf16), both K-major (bits 15, 16 = 0),
 // N >> 3 (bits 17-22), M >> 4 (bits 24-28).
-uint32_t make_idesc(int in_dtype, int bn) {
+uint32_t make_idesc(int in_dtype, int bm, int bn) {
     const uint32_t fmt = in_dtype == MR_BF16 ? 1u : 0u;
-    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(bm >> 4) << 24);
 }
 
 // Tile selection: estimated time = waves x k-blocks x the tile's time per
@@ -508,9 +517,11 @@ uint32_t make_idesc(int in_dtype, int bn) {
 // wave, and these are those costs / 40 k-blocks.  Narrow tiles are cheap per
 // wave (two k-blocks per ring stage, short MMAs) but need more waves; wide
 // tiles reuse each A stage over more columns but run longer per wave.  Row
-// tails count as whole 128-row tiles, so an M with a small M % 128 pays for
-// the padding it creates (the audit's tail-tile rule, restated as waves over
-// 148 SMs); the narrow N = 96 projections favour spreading tiles over SMs.
+// tails count as whole tiles, so an M with a small M % 128 pays for the
+// padding it creates, and a 64-row tile (half the padding, tcgen05 M = 64)
+// wins where that padding costs a wave (the audit's tail-tile rule,
+// restated as waves over 148 SMs); the narrow N = 96 projections favour
+// spreading tiles over SMs.
 // Groups packed per tile of width bn: a tile holds whole groups when N
 // divides bn and is a multiple of 16 (so no 16-column chunk straddles two
 // groups); otherwise 1 (a group spans ceil(N / bn) tiles).
@@ -525,15 +536,19 @@ int64_t n_slots(int bn, int N, int G, int P) {
 
 int select_tile_grouped(int M, int N, int K, int G, int sms) {
     if (M < 1 || N < 1 || K < 1 || G < 1 || sms < 1) return -1;
-    // ns per k-block of one tile, for BN = 32, 64, 96, 128, 192, 256.
-    const double kb_ns[kNumTiles] = {175.0, 193.0, 225.0, 254.0, 338.0, 438.0};
+    // ns per k-block of one tile: 128 x (32, 64, 96, 128, 192, 256), then
+    // 64 x (128, 256).  The 64-row tiles measured 0.78x the 128 x 128 and
+    // 0.85x the 128 x 256 per-wave cost in the same all-tiles study, and are
+    // placed at those ratios.
+    const double kb_ns[kNumTiles] = {175.0, 193.0, 225.0, 254.0, 338.0, 438.0, 198.0, 372.0};
     const int64_t nkb = (K + BK - 1) / BK;
     int best = -1;
     double best_t = 1e300;
     for (int t = 0; t < kNumTiles; ++t) {
         const int bn = kTiles[t].bn;
         const int P = pack_factor(bn, N, G);
-        const int64_t tiles = (int64_t)((M + BM - 1) / BM) * n_slots(bn, N, G, P);
+        const int bm = kTiles[t].bm;
+        const int64_t tiles = (int64_t)((M + bm - 1) / bm) * n_slots(bn, N, G, P);
         const int64_t waves = (tiles + sms - 1) / sms;
         const double t_est = (double)waves * (double)nkb * kb_ns[t];
         if (t_est < best_t * 0.999) {
@@ -586,19 +601,19 @@ mr_status launch(const void *A, int64_t lda, const void *const *Wts, int64_t ldw
     args.G = G;
     args.ldc = ldc;
     args.raster = raster;
-    args.idesc = make_idesc(in_dtype, td.bn);
-    if (!encode_operand(&args.tmA, A, M, K, lda, in_dtype, BM)) return MR_ERR_CUDA;
+    args.idesc = make_idesc(in_dtype, td.bm, td.bn);
+    if (!encode_operand(&args.tmA, A, M, K, lda, in_dtype, td.bm)) return MR_ERR_CUDA;
     const int b_rows = args.P > 1 ? N : td.bn;
     for (int g = 0; g < G; ++g) {
         if (!encode_operand(&args.tmB[g], Wts[g], N, K, ldw, in_dtype, b_rows)) return MR_ERR_CUDA;
         args.C[g] = Cs[g];
     }
 
-    const int64_t ntiles = (int64_t)args.ntn * ((M + BM - 1) / BM);
+    const int64_t ntiles = (int64_t)args.ntn * ((M + td.bm - 1) / td.bm);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)std::min<int64_t>(ntiles, sms));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem_bytes_for(td.bn, td.stages);
+    cfg.dynamicSmemBytes = smem_bytes_for(td.bm, td.bn, td.stages);
     cfg.stream = static_cast<cudaStream_t>(stream);
     e = cudaLaunchKernelEx(&cfg, kernel_for<MAXG>(t, out_dtype), args);
     return mr_host::cuda_status(e);
