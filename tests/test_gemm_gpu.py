@@ -113,7 +113,7 @@ def test_chunk_small_full_parity_all_dtypes():
 def test_edges(M, N, K):
     a = synth.normal_bits(11 + M, (M, K), "f16", 1.0)
     w = synth.normal_bits(12 + N, (N, K), "f16", 1.0 / np.sqrt(K))
-    for tile in (-1, 0, 5, 6, 7):
+    for tile in (-1, 0, 5, 6, 7, 8):
         c, _ = run_gemm(a, w, tile=tile)
         check(c, a, w, "f16", "f16")
 
@@ -135,7 +135,7 @@ def test_bitwise_identical_across_tiles_M_and_row_order(M, N, fmt):
     _, auto = run_gemm(a, w, in_fmt=fmt, out_fmt=fmt)
     assert np.array_equal(auto, ref)
     for m in (1, 64, 127, 129, M // 2):
-        for tile in (3, 6):   # a 128-row and a 64-row tile
+        for tile in (3, 6, 8):   # a 128-row, a 64-row and the two-CTA 256-row tile
             _, part = run_gemm(a[:m], w, in_fmt=fmt, out_fmt=fmt, tile=tile)
             assert np.array_equal(part, ref[:m]), f"prefix M={m} differs (tile {tile})"
     perm = np.random.default_rng(5).permutation(M)

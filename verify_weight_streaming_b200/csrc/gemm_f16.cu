@@ -55,6 +55,7 @@ struct TileDesc {
     int acc_cols;   // tensor-memory columns per accumulator buffer (power of two >= bn)
     int kpb;        // k-blocks per ring stage (one barrier wait and one commit each)
     const char *name;
+    bool pair = false;  // two CTAs per tile (cta_group::2): bm = 256, 128 rows per CTA
 };
 
 // Tiles up to BN = 128 take two k-blocks per ring stage: their MMAs are short
@@ -66,6 +67,7 @@ constexpr TileDesc kTiles[] = {
     {128, 32, 8, 32, 2, "128x32"},   {128, 64, 8, 64, 2, "128x64"},   {128, 96, 7, 128, 2, "128x96"},
     {128, 128, 6, 128, 2, "128x128"}, {128, 192, 5, 256, 1, "128x192"}, {128, 256, 4, 256, 1, "128x256"},
     {64, 128, 8, 128, 2, "64x128"},   {64, 256, 5, 256, 1, "64x256"},
+    {256, 256, 7, 256, 1, "256x256", true},
 };
 constexpr int kNumTiles = sizeof(kTiles) / sizeof(kTiles[0]);
 
@@ -139,6 +141,75 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+// ---- CTA-pair (cta_group::2) helpers -------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// The shared::cluster address of the same offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+
+// Every thread of both CTAs: arrive (release) and wait (acquire) on the cluster barrier.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// One MMA for the pair: M = 256 (128 rows of A from each CTA's shared
+// memory), N columns (N / 2 rows of Wt from each CTA), K = 16; the
+// accumulator's rows 128v..128v+127 land in CTA v's tensor memory.
+__device__ __forceinline__ void mma_f16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on the barrier at this offset in both CTAs of the pair once every
+// tcgen05 operation issued so far by this thread completes.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    const uint16_t both = 0x3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"(both)
+        : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on a
+// barrier of either CTA of the pair (cluster address).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                                 uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster)
         : "memory");
 }
 
@@ -425,6 +496,191 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
 }
 
+// ---- the CTA-pair kernel: 256 x 256 tiles on two SMs (cta_group::2) ---------
+//
+// A cluster of two CTAs computes a 256 x 256 output tile with one
+// tcgen05.mma.cta_group::2 per K step of 16: CTA v loads rows 128v..128v+127
+// of the tile's A block and rows 128v..128v+127 of its Wt block (columns of
+// the output) into its own shared memory, and CTA v's tensor memory receives
+// rows 128v..128v+127 of the accumulator.  Each CTA streams 32 KB per
+// k-block instead of the 48 KB a 128 x 256 tile needs.  The leader (rank 0)
+// issues every MMA from one elected thread and waits on its own full
+// barriers, which count the TMA bytes of both CTAs (the peer's loads signal
+// the leader's barrier; no load is multicast); its commits arrive on the
+// barriers of both CTAs.  Both CTAs' epilogue warps release an accumulator
+// buffer on the leader's barrier.  The K sequence is that of every other
+// tile, so the bits are too.
+constexpr int kPairN = 256;          // output columns per tile
+constexpr int kPairRows = 256;       // output rows per tile (128 per CTA)
+constexpr int kPairStages = 7;       // k-blocks of 32 KB per CTA
+
+__host__ __device__ constexpr uint32_t pair_smem_bytes() {
+    return (uint32_t)kPairStages * (a_bytes_for(128) + (uint32_t)(kPairN / 2) * BK * 2) + 1024 + 256;
+}
+
+template <int OUT, int MAXG>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ GemmArgs<MAXG> args) {
+    constexpr int BMH = kPairRows / 2;                 // A rows per CTA
+    constexpr int BNH = kPairN / 2;                    // Wt rows per CTA
+    constexpr uint32_t kAB = (uint32_t)BMH * BK * 2;   // 16 KB
+    constexpr uint32_t kBB = (uint32_t)BNH * BK * 2;   // 16 KB
+    constexpr int NST = kPairStages;
+    static_assert(NST >= kProducers, "ring too short for the producer warps");
+    constexpr uint32_t ACC_COLS = kPairN;
+    constexpr uint32_t kTmemCols = 2 * ACC_COLS;
+    const CUtensorMap &tmA = args.tmA;
+    const int M = args.M, N = args.N, K = args.K;
+    const int64_t ldc = args.ldc;
+    const uint32_t idesc = args.idesc;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+    const uint32_t sA = base;
+    const uint32_t sB = base + NST * kAB;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + NST * (kAB + kBB));
+    uint64_t *full = bars;                  // [NST] TMA (both CTAs) -> MMA; used in the leader
+    uint64_t *empty = bars + NST;           // [NST] MMA -> this CTA's producers
+    uint64_t *acc_full = bars + 2 * NST;    // [2] MMA -> this CTA's epilogue
+    uint64_t *acc_empty = bars + 2 * NST + 2;  // [2] both epilogues -> MMA; used in the leader
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * NST + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int ntn = args.ntn;
+    const int ntm = (M + kPairRows - 1) / kPairRows;
+    const int ntiles = ntm * ntn;
+    const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+    const int nkb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < NST; ++st) {
+            mbar_init(smem_u32(&full[st]), 1);
+            mbar_init(smem_u32(&empty[st]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&acc_full[b]), 1);
+            mbar_init(smem_u32(&acc_empty[b]), 8);  // four epilogue warps in each CTA
+        }
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        if (MAXG == 1) prefetch_tmap(&args.tmB[0]);
+    }
+    if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers initialised, tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0 || warp == 6) {
+        // Producers of this CTA's halves; the leader's thread also arms the
+        // leader's full barrier with the bytes of both CTAs.
+        const uint32_t pidx = warp == 0 ? 0u : 1u;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = pair; t < ntiles && ok; t += npairs) {
+            int mt, slot;
+            tile_coords(t, ntm, ntn, args.raster, mt, slot);
+            const int m0 = mt * kPairRows + (int)rank * BMH;
+            const int g = slot / args.tn_per_group;
+            const int n0 = (slot % args.tn_per_group) * kPairN + (int)rank * BNH;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                if (it % kProducers != pidx) continue;
+                const uint32_t st = it % NST;
+                const uint32_t par = ((it / NST) & 1u) ^ 1u;
+                ok = mbar_wait_bounded(smem_u32(&empty[st]), par, MR_DEVERR_GEMM_TIMEOUT);
+                if (!ok) break;
+                if (lane == 0) {
+                    const uint32_t fb = map_to_rank(smem_u32(&full[st]), 0u);
+                    if (leader) mbar_arrive_expect_tx(smem_u32(&full[st]), 2u * (kAB + kBB));
+                    tma_load_2d_pair(sA + st * kAB, &tmA, kb * BK, m0, fb);
+                    tma_load_2d_pair(sB + st * kBB, &args.tmB[g], kb * BK, n0, fb);
+                }
+                __syncwarp();
+            }
+        }
+        // Tail: wait until the MMAs have released the last fill of every stage
+        // this producer wrote, so that no commit arrives on this CTA's
+        // barriers after it exits.
+        for (uint32_t j = it > (uint32_t)NST ? it - NST : 0u; j < it && ok; ++j) {
+            if (j % kProducers != pidx) continue;
+            ok = mbar_wait_bounded(smem_u32(&empty[j % NST]), (j / NST) & 1u, MR_DEVERR_GEMM_TIMEOUT);
+        }
+    } else if (warp == 1) {
+        if (leader) {
+            const uint64_t adesc0 = sw128_desc(sA), bdesc0 = sw128_desc(sB);
+            const bool issuer = elect_one();
+            uint32_t it = 0, ti = 0;
+            bool ok = true;
+            for (int t = pair; t < ntiles && ok; t += npairs, ++ti) {
+                const uint32_t b = ti & 1u;
+                ok = mbar_wait_bounded(smem_u32(&acc_empty[b]), ((ti >> 1) & 1u) ^ 1u, MR_DEVERR_GEMM_TIMEOUT);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t acc = tmem + b * ACC_COLS;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const uint32_t st = it % NST;
+                    ok = mbar_wait_bounded(smem_u32(&full[st]), (it / NST) & 1u, MR_DEVERR_GEMM_TIMEOUT);
+                    if (!ok) break;
+                    tc_fence_after();
+                    __syncwarp();
+                    if (issuer) {
+                        // K steps of 16 in ascending order, as in every tile.
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t ad = adesc0 + (uint64_t)((st * kAB + kk * 32) >> 4);
+                            const uint64_t bd = bdesc0 + (uint64_t)((st * kBB + kk * 32) >> 4);
+                            mma_f16_pair(acc, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                        mma_commit_pair(smem_u32(&empty[st]));
+                    }
+                    __syncwarp();
+                }
+                if (ok && issuer) mma_commit_pair(smem_u32(&acc_full[b]));
+                __syncwarp();
+            }
+        }
+    } else {
+        // Epilogue warps 2..5 of both CTAs: warp w reads tensor-memory lanes
+        // 32*(w%4) .. +31 of this CTA's half, rows 128 * rank + 32 * (w%4) ...
+        const int q = warp & 3;
+        uint32_t ti = 0;
+        for (int t = pair; t < ntiles; t += npairs, ++ti) {
+            const uint32_t b = ti & 1u;
+            int mt, slot;
+            tile_coords(t, ntm, ntn, args.raster, mt, slot);
+            const int g = slot / args.tn_per_group;
+            const int n0 = (slot % args.tn_per_group) * kPairN;
+            const int row = mt * kPairRows + (int)rank * BMH + 32 * q + lane;
+            if (!mbar_wait_bounded(smem_u32(&acc_full[b]), (ti >> 1) & 1u, MR_DEVERR_GEMM_TIMEOUT)) break;
+            tc_fence_after();
+            const uint32_t acc = tmem + b * ACC_COLS + ((uint32_t)(32 * q) << 16);
+#pragma unroll 1
+            for (int c = 0; c < kPairN / 16; ++c) {
+                uint32_t r[16];
+                tmem_ld16(acc + (uint32_t)(c * 16), r);
+                const int col = n0 + c * 16;
+                if (row < M && col < N) store16<OUT>(args.C[g], ldc, row, col, N, r);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&acc_empty[b]), 0u));
+        }
+    }
+
+    // Neither CTA frees tensor memory or exits while its pair may still use it.
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
 // ---- host side -------------------------------------------------------------
 
 constexpr int kMaxGroups = 64;
@@ -439,6 +695,7 @@ constexpr KernelFn<MAXG> kernel_of() {
 
 template <int OUT, int MAXG>
 KernelFn<MAXG> pick_out(int t) {
+    if (kTiles[t].pair) return gemm_pair_kernel<OUT, MAXG>;
     switch (t) {
         case 0: return kernel_of<0, OUT, MAXG>();
         case 1: return kernel_of<1, OUT, MAXG>();
@@ -449,6 +706,41 @@ KernelFn<MAXG> pick_out(int t) {
         case 6: return kernel_of<6, OUT, MAXG>();
         default: return kernel_of<7, OUT, MAXG>();
     }
+}
+
+// Dynamic shared memory of tile t's kernel.
+uint32_t tile_smem_bytes(int t) {
+    const TileDesc &td = kTiles[t];
+    return td.pair ? pair_smem_bytes() : smem_bytes_for(td.bm, td.bn, td.stages);
+}
+
+// Clusters of two CTAs of the pair kernel that fit on the device at once
+// (both SMs of a pair must sit in one GPC), or 0 when the query fails.
+int max_pairs(int device) {
+    static std::mutex m;
+    static int cached[64] = {};
+    std::lock_guard<std::mutex> lock(m);
+    if (device < 0 || device >= 64) return 0;
+    if (cached[device] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = pair_smem_bytes();
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<MR_F16, 1>, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            return 0;
+        }
+        cached[device] = n;
+    }
+    return cached[device];
 }
 
 template <int MAXG>
@@ -475,7 +767,7 @@ cudaError_t init_device(int device) {
     if (device >= 0 && device < 64 && !g_attr_done[device]) {
         for (int t = 0; t < kNumTiles; ++t)
             for (int out = 0; out < 3; ++out) {
-                const int smem = (int)smem_bytes_for(kTiles[t].bm, kTiles[t].bn, kTiles[t].stages);
+                const int smem = (int)tile_smem_bytes(t);
                 cudaError_t e = cudaFuncSetAttribute(kernel_for<1>(t, out),
                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
                 if (e != cudaSuccess) return e;
@@ -525,8 +817,8 @@ uint32_t make_idesc(int in_dtype, int bm, int bn) {
 // Groups packed per tile of width bn: a tile holds whole groups when N
 // divides bn and is a multiple of 16 (so no 16-column chunk straddles two
 // groups); otherwise 1 (a group spans ceil(N / bn) tiles).
-int pack_factor(int bn, int N, int G) {
-    if (G > 1 && N < bn && bn % N == 0 && N % 16 == 0) return bn / N;
+int pack_factor(int bn, int N, int G, bool pair = false) {
+    if (!pair && G > 1 && N < bn && bn % N == 0 && N % 16 == 0) return bn / N;
     return 1;
 }
 
@@ -534,22 +826,28 @@ int64_t n_slots(int bn, int N, int G, int P) {
     return P > 1 ? (int64_t)((G + P - 1) / P) : (int64_t)G * ((N + bn - 1) / bn);
 }
 
-int select_tile_grouped(int M, int N, int K, int G, int sms) {
+int select_tile_grouped(int M, int N, int K, int G, int sms, int pairs) {
     if (M < 1 || N < 1 || K < 1 || G < 1 || sms < 1) return -1;
     // ns per k-block of one tile: 128 x (32, 64, 96, 128, 192, 256), then
     // 64 x (128, 256).  The 64-row tiles measured 0.78x the 128 x 128 and
     // 0.85x the 128 x 256 per-wave cost in the same all-tiles study, and are
     // placed at those ratios.
-    const double kb_ns[kNumTiles] = {175.0, 193.0, 225.0, 254.0, 338.0, 438.0, 198.0, 372.0};
+    // The 256 x 256 pair tile runs one tile per two SMs; it measured 0.96x
+    // the 128 x 256 tile's cost per wave (a wave of pairs covers the same
+    // output area as a wave of 128 x 256 tiles).
+    const double kb_ns[kNumTiles] = {175.0, 193.0, 225.0, 254.0, 338.0, 438.0, 198.0, 372.0, 420.0};
     const int64_t nkb = (K + BK - 1) / BK;
     int best = -1;
     double best_t = 1e300;
     for (int t = 0; t < kNumTiles; ++t) {
         const int bn = kTiles[t].bn;
-        const int P = pack_factor(bn, N, G);
+        const bool pair = kTiles[t].pair;
+        if (pair && pairs < 1) continue;
+        const int P = pack_factor(bn, N, G, pair);
         const int bm = kTiles[t].bm;
         const int64_t tiles = (int64_t)((M + bm - 1) / bm) * n_slots(bn, N, G, P);
-        const int64_t waves = (tiles + sms - 1) / sms;
+        const int64_t slots = pair ? pairs : sms;
+        const int64_t waves = (tiles + slots - 1) / slots;
         const double t_est = (double)waves * (double)nkb * kb_ns[t];
         if (t_est < best_t * 0.999) {
             best_t = t_est;
@@ -559,7 +857,7 @@ int select_tile_grouped(int M, int N, int K, int G, int sms) {
     return best;
 }
 
-int select_tile(int M, int N, int K, int sms) { return select_tile_grouped(M, N, K, 1, sms); }
+int select_tile(int M, int N, int K, int sms, int pairs) { return select_tile_grouped(M, N, K, 1, sms, pairs); }
 
 // Validate, encode the tensor maps and launch one grouped GEMM.
 template <int MAXG>
@@ -586,13 +884,15 @@ mr_status launch(const void *A, int64_t lda, const void *const *Wts, int64_t ldw
     e = init_device(device);
     if (e != cudaSuccess) return MR_ERR_CUDA;
     const int sms = mr_host::sm_count() > 0 ? mr_host::sm_count() : 148;
-    const int t = tile_id >= 0 ? tile_id : select_tile_grouped(M, N, K, G, sms);
+    const int pairs = max_pairs(device);
+    const int t = tile_id >= 0 ? tile_id : select_tile_grouped(M, N, K, G, sms, pairs);
     if (t < 0) return MR_ERR_INVALID_ARG;
     const TileDesc &td = kTiles[t];
+    if (td.pair && pairs < 1) return MR_ERR_UNSUPPORTED;
 
     GemmArgs<MAXG> args;
     memset(&args, 0, sizeof(args));
-    args.P = pack_factor(td.bn, N, G);
+    args.P = pack_factor(td.bn, N, G, td.pair);
     args.tn_per_group = (N + td.bn - 1) / td.bn;
     args.ntn = (int)n_slots(td.bn, N, G, args.P);
     args.M = M;
@@ -602,8 +902,9 @@ mr_status launch(const void *A, int64_t lda, const void *const *Wts, int64_t ldw
     args.ldc = ldc;
     args.raster = raster;
     args.idesc = make_idesc(in_dtype, td.bm, td.bn);
-    if (!encode_operand(&args.tmA, A, M, K, lda, in_dtype, td.bm)) return MR_ERR_CUDA;
-    const int b_rows = args.P > 1 ? N : td.bn;
+    // The pair tile's CTAs each load 128 rows of A and bn / 2 rows of Wt.
+    if (!encode_operand(&args.tmA, A, M, K, lda, in_dtype, td.pair ? td.bm / 2 : td.bm)) return MR_ERR_CUDA;
+    const int b_rows = args.P > 1 ? N : (td.pair ? td.bn / 2 : td.bn);
     for (int g = 0; g < G; ++g) {
         if (!encode_operand(&args.tmB[g], Wts[g], N, K, ldw, in_dtype, b_rows)) return MR_ERR_CUDA;
         args.C[g] = Cs[g];
@@ -611,9 +912,10 @@ mr_status launch(const void *A, int64_t lda, const void *const *Wts, int64_t ldw
 
     const int64_t ntiles = (int64_t)args.ntn * ((M + td.bm - 1) / td.bm);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)std::min<int64_t>(ntiles, sms));
+    cfg.gridDim = td.pair ? dim3((unsigned)(2 * std::min<int64_t>(ntiles, pairs)))
+                          : dim3((unsigned)std::min<int64_t>(ntiles, sms));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem_bytes_for(td.bm, td.bn, td.stages);
+    cfg.dynamicSmemBytes = tile_smem_bytes(t);
     cfg.stream = static_cast<cudaStream_t>(stream);
     e = cudaLaunchKernelEx(&cfg, kernel_for<MAXG>(t, out_dtype), args);
     return mr_host::cuda_status(e);
@@ -629,10 +931,23 @@ extern "C" const char *gemm_f16_tile_name(int32_t tile_id) {
     return mr::gemm::kTiles[tile_id].name;
 }
 
-extern "C" int32_t gemm_f16_select_tile(int32_t M, int32_t N, int32_t K) {
-    int sms = mr_host::sm_count();
+namespace mr {
+namespace gemm {
+// SMs and CTA pairs of the current device (148 and 74 when no device answers).
+void device_slots(int &sms, int &pairs) {
+    sms = mr_host::sm_count();
     if (sms <= 0) sms = 148;
-    return mr::gemm::select_tile(M, N, K, sms);
+    int device = 0;
+    pairs = (cudaGetDevice(&device) == cudaSuccess && init_device(device) == cudaSuccess) ? max_pairs(device) : 0;
+    if (pairs <= 0) pairs = sms / 2;
+}
+}  // namespace gemm
+}  // namespace mr
+
+extern "C" int32_t gemm_f16_select_tile(int32_t M, int32_t N, int32_t K) {
+    int sms, pairs;
+    mr::gemm::device_slots(sms, pairs);
+    return mr::gemm::select_tile(M, N, K, sms, pairs);
 }
 
 extern "C" mr_status gemm_f16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw, void *C, int64_t ldc,
@@ -659,7 +974,7 @@ extern "C" mr_status gemm_f16_grouped(const void *A, int64_t lda, const void *co
 }
 
 extern "C" int32_t gemm_f16_grouped_select_tile(int32_t M, int32_t N, int32_t K, int32_t G) {
-    int sms = mr_host::sm_count();
-    if (sms <= 0) sms = 148;
-    return mr::gemm::select_tile_grouped(M, N, K, G, sms);
+    int sms, pairs;
+    mr::gemm::device_slots(sms, pairs);
+    return mr::gemm::select_tile_grouped(M, N, K, G, sms, pairs);
 }
