@@ -3,9 +3,10 @@
 One step = one pass of the router hot path over one batch: for each window
 size m in (1, 2, 4, 8, 16), A[m,2560] bf16 x W_r[2560,512] bf16 -> fp32 logits
 (weight streamed once) -> per-row top-10.  That is 31 rows per step.  The
-reported value is the two-launch form (mrgemv_bf16 then router_topk per
-window); the fused form (router_gemv_topk, one launch per window) is timed
-over the same K steps and printed beside it.  The weight comes from a
+reported value is the two-launch form (one router_gemv_topk call per window
+with MR_ROUTER_TWO_LAUNCH: the GEMV kernel, then the top-k kernel); the fused
+form (one launch per window) is timed over the same K steps and printed
+beside it.  The weight comes from a
 rotating pool of copies larger than twice the L2, so every launch reads it
 from HBM.
 
@@ -297,16 +298,13 @@ class RouterBench:
         return w
 
     def step(self, flags, fused=True):
-        """One router step: for each window size, GEMV + top-10 (one fused launch,
-        or the two-launch form mrgemv_bf16 then router_topk)."""
+        """One router step: for each window size, GEMV + top-10 in one
+        router_gemv_topk call (one fused launch, or the GEMV kernel then the
+        top-k kernel with MR_ROUTER_TWO_LAUNCH)."""
         mr = self.mr
         for m in WINDOWS:
-            if fused:
-                mr.router_gemv_topk(self.A[:m], self._next_w(), TOPK, self.idx[m], self.val[m],
-                                    workspace=self.ws, flags=flags)
-            else:
-                mr.mrgemv_bf16(self.A[:m], self._next_w(), self.C[m], flags=flags)
-                mr.router_topk(self.C[m], TOPK, self.idx[m], self.val[m])
+            mr.router_gemv_topk(self.A[:m], self._next_w(), TOPK, self.idx[m], self.val[m],
+                                workspace=self.ws, flags=flags if fused else flags | mr.MR_ROUTER_TWO_LAUNCH)
 
     def capture_steps(self, count, flags, fused=True):
         """One CUDA graph per step, each with its own slice of the weight pool."""
@@ -348,9 +346,8 @@ def run_gpu(args, world, rank, local):
     rb = RouterBench(device)
     flags = 0 if args.no_pdl else mr.MR_GEMV_PDL
     steps_per_cycle = max(1, rb.pool // len(WINDOWS))
-    # Two public forms of the router step give identical outputs: two launches
-    # per window (mrgemv_bf16, then router_topk) and one fused launch
-    # (router_gemv_topk).  `value` is always the two-launch form; the fused
+    # Two forms of the router step give identical outputs: two launches per
+    # window (the GEMV kernel, then the top-k kernel) and one fused launch.  `value` is always the two-launch form; the fused
     # form is timed over the same K steps and printed beside it (on B200 its
     # cross-CTA ticket and generation handshake costs more than the kernel
     # boundary it removes).
@@ -590,11 +587,8 @@ def run_e2e(rb, args, world, device, fused=True):
         a_dev.copy_(a_host, non_blocking=True)
         for m in WINDOWS:
             a_m, idx_m, val_m = views[m]
-            if fused:
-                mr.router_gemv_topk(a_m, rb._next_w(), TOPK, idx_m, val_m, workspace=rb.ws, flags=flags)
-            else:
-                mr.mrgemv_bf16(a_m, rb._next_w(), rb.C[m], flags=flags)
-                mr.router_topk(rb.C[m], TOPK, idx_m, val_m)
+            mr.router_gemv_topk(a_m, rb._next_w(), TOPK, idx_m, val_m, workspace=rb.ws,
+                                flags=flags if fused else flags | mr.MR_ROUTER_TWO_LAUNCH)
         out_host.copy_(out_dev, non_blocking=True)
 
     with torch.cuda.stream(rb.stream):
@@ -654,8 +648,8 @@ def run_e2e(rb, args, world, device, fused=True):
     d2h = sum(m * TOPK * 8 for m in WINDOWS)
     return {"value": us / (steps * step_rows() * world), "unit": "us/row",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "api": ("router_gemv_topk" if fused else "mrgemv_bf16 + router_topk")
-                   + " (verify_weight_streaming_b200), pinned host buffers",
+            "api": "router_gemv_topk" + ("" if fused else " with MR_ROUTER_TWO_LAUNCH (GEMV kernel + top-k kernel)")
+                   + " (verify_weight_streaming_b200), one call per window, pinned host buffers",
             "graph_value": (graph_us / (steps * step_rows() * world)) if graph_us is not None else None,
             "results_ok": results_ok,
             "graph_note": "same calls and host copies, captured once into a CUDA graph and replayed"}

@@ -137,6 +137,14 @@ mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t flags, int3
  *          run at the same time (other streams) need separate workspaces.
  */
 #define MR_ROUTER_TICKET_BYTES 256u
+/*
+ * MR_ROUTER_TWO_LAUNCH (flag of router_gemv_topk / _noalloc): run the window
+ * as the GEMV kernel followed by the router_topk kernel (programmatic
+ * dependent launch) instead of one fused launch: the same outputs, bit for
+ * bit, from one call.  The logits go to `logits`, or to the workspace past
+ * its ticket block; the ticket block is not used.
+ */
+#define MR_ROUTER_TWO_LAUNCH 0x4u
 mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt, int64_t ldw,
                            float *logits, int64_t ldl, int32_t m, int32_t n, int32_t k,
                            int32_t topk, int32_t *idx, float *val, int64_t ldo,
@@ -162,7 +170,8 @@ size_t router_gemv_topk_workspace_bytes(int32_t m, int32_t n, int32_t logits_pro
  * The call allocates nothing: its first call on a device looks up the array's
  * device address (cudaGetSymbolAddress) with that device current, so make
  * that first call before any stream capture.  Each call clears the ticket on
- * `stream` (cudaMemsetAsync) and then launches.  Every call shares the one
+ * `stream` (cudaMemsetAsync; not with MR_ROUTER_TWO_LAUNCH, which uses no
+ * ticket) and then launches.  Every call shares the one
  * array, so calls that overlap on the GPU (other streams, or overlapping
  * launches) race and must not be issued.
  */

@@ -104,3 +104,28 @@ def test_many_calls_graph_and_pdl_reuse_one_workspace():
     for (c, ir, vr), (i, v) in zip(refs, outs):
         assert np.array_equal(host(i), ir)
     assert int(host(ws)[0]) == 0
+
+
+@pytest.mark.parametrize("m", [1, 5, 16])
+@pytest.mark.parametrize("with_logits", [True, False])
+def test_two_launch_flag_matches_fused_and_separate_calls(m, with_logits):
+    """MR_ROUTER_TWO_LAUNCH: one call, GEMV kernel then top-k kernel: the same bits."""
+    a, w = synth.router(m)
+    A, W = dev_bits(a), dev_bits(w)
+    c_ref, i_ref, v_ref = two_launch(A, W, m, 512, 10)
+    ws = workspace(m, 512, with_logits)
+    ws.fill_(-1)   # the ticket block is not used by this form
+    idx = torch.full((m, 10), -1, dtype=torch.int32, device="cuda")
+    val = torch.full((m, 10), float("nan"), dtype=torch.float32, device="cuda")
+    logits = torch.empty((m, 512), dtype=torch.float32, device="cuda") if with_logits else None
+    mr.router_gemv_topk(A, W, 10, idx, val, logits=logits, workspace=ws,
+                        flags=mr.MR_GEMV_PDL | mr.MR_ROUTER_TWO_LAUNCH)
+    assert np.array_equal(host(idx), i_ref)
+    assert np.array_equal(host(val).view(np.uint32), v_ref.view(np.uint32))
+    if with_logits:
+        assert np.array_equal(host(logits).view(np.uint32), c_ref.view(np.uint32))
+    else:
+        got = host(ws)[64:64 + m * 512].view(np.float32).reshape(m, 512)
+        assert np.array_equal(got.view(np.uint32), c_ref.view(np.uint32))
+    with pytest.raises(mr.MrError):
+        mr.router_gemv_topk(A, W, 10, idx, val, workspace=ws, flags=mr.MR_GEMV_SIGMOID)

@@ -18,6 +18,7 @@ MR_OK, MR_ERR_INVALID_ARG, MR_ERR_MISALIGNED, MR_ERR_UNSUPPORTED, MR_ERR_CUDA, M
 MR_F16, MR_BF16, MR_F32 = 0, 1, 2
 MR_GEMV_PDL = 0x1
 MR_GEMV_SIGMOID = 0x2
+MR_ROUTER_TWO_LAUNCH = 0x4
 MR_DEVERR_GEMV_TIMEOUT, MR_DEVERR_GEMM_TIMEOUT, MR_DEVERR_TOPK_TIMEOUT, MR_DEVERR_SELFTEST = 1, 2, 4, 8
 
 EXPORTS = (

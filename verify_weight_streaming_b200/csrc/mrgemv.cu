@@ -835,16 +835,33 @@ mr_status prepare_router(const void *A, int64_t lda, const void *Wt, int64_t ldw
 }  // namespace gemv
 }  // namespace mr
 
+namespace mr {
+namespace gemv {
+
+// The fused launch, or (MR_ROUTER_TWO_LAUNCH) the GEMV kernel then the top-k
+// kernel on the same logits; every argument is checked before either.
+mr_status launch_router(const Params &p, const Plan &pl, uint32_t flags, void *stream) {
+    const uint32_t gemv_flags = flags & ~MR_ROUTER_TWO_LAUNCH;
+    if (!(flags & MR_ROUTER_TWO_LAUNCH)) return enqueue(p, pl, gemv_flags, true, stream);
+    const mr_status st = enqueue(p, pl, gemv_flags, false, stream);
+    if (st != MR_OK) return st;
+    return router_topk_ex(p.C, p.ldc, p.m, p.n, p.topk, p.idx, p.val, p.ldo, 0, stream);
+}
+
+}  // namespace gemv
+}  // namespace mr
+
 extern "C" mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *logits,
                                       int64_t ldl, int32_t m, int32_t n, int32_t k, int32_t topk, int32_t *idx,
                                       float *val, int64_t ldo, void *workspace, size_t workspace_bytes,
                                       uint32_t flags, void *stream) {
+    if (flags & ~(MR_GEMV_PDL | MR_ROUTER_TWO_LAUNCH)) return MR_ERR_INVALID_ARG;
     mr::gemv::Params p;
     mr::gemv::Plan pl;
     const mr_status st = mr::gemv::prepare_router(A, lda, Wt, ldw, logits, ldl, m, n, k, topk, idx, val, ldo,
-                                                  workspace, workspace_bytes, flags, p, pl);
+                                                  workspace, workspace_bytes, flags & ~MR_ROUTER_TWO_LAUNCH, p, pl);
     if (st != MR_OK) return st;
-    return mr::gemv::enqueue(p, pl, flags, true, stream);
+    return mr::gemv::launch_router(p, pl, flags, stream);
 }
 
 extern "C" mr_status mrgemv_bf16(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *C,
@@ -904,13 +921,15 @@ extern "C" mr_status router_gemv_topk_noalloc(const void *A, int64_t lda, const 
     mr_status st = mr::gemv::noalloc_scratch(&scratch);
     if (st != MR_OK) return st;
     // Every argument is checked before anything is put on the stream.
+    if (flags & ~(MR_GEMV_PDL | MR_ROUTER_TWO_LAUNCH)) return MR_ERR_INVALID_ARG;
     mr::gemv::Params p;
     mr::gemv::Plan pl;
     st = mr::gemv::prepare_router(A, lda, Wt, ldw, logits, ldl, m, n, k, topk, idx, val, ldo, scratch,
-                                  mr::gemv::kNoAllocScratchBytes, flags, p, pl);
+                                  mr::gemv::kNoAllocScratchBytes, flags & ~MR_ROUTER_TWO_LAUNCH, p, pl);
     if (st != MR_OK) return st;
     // The array keeps whatever the last call left; the ticket must start at zero.
-    if (cudaMemsetAsync(scratch, 0, MR_ROUTER_TICKET_BYTES, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (!(flags & MR_ROUTER_TWO_LAUNCH) &&
+        cudaMemsetAsync(scratch, 0, MR_ROUTER_TICKET_BYTES, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return MR_ERR_CUDA;
-    return mr::gemv::enqueue(p, pl, flags, true, stream);
+    return mr::gemv::launch_router(p, pl, flags, stream);
 }
