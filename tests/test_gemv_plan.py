@@ -31,7 +31,11 @@ def test_plan_invariants(flags):
     ks = [8, 64, 136, 896, 1024, 2048, 2560, 4088, 4096]
     for m, n, k in itertools.product(ms, ns, ks):
         p = mr.mrgemv_bf16_plan(m, n, k, flags, SMS, OPTIN)
-        assert 1 <= p["grid"] <= min(SMS, n)
+        assert 1 <= p["grid"] <= min(SMS, n) or (flags and p["grid"] == 2 * SMS <= n)
+        if p["grid"] > SMS:
+            # two CTAs per SM: each fits half of the SM's shared memory and
+            # registers (at most 128 a thread), and only small row buckets split
+            assert p["smem_bytes"] <= 110 * 1024 and p["threads"] <= 256 and p["row_bucket"] <= 4
         # 16 warps at most (every kernel is built for 512 threads of <= 128 registers)
         assert p["threads"] == 32 * p["k_warps"] * p["column_warps"] <= 32 * 16
         assert p["smem_bytes"] <= OPTIN

@@ -642,18 +642,29 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     pl.CG = col_group_rt(pl.MB, k);
     pl.KW = k_warps(k);
     pl.G = std::min(sms, n);
+    constexpr size_t kPdlBudget = 110 * 1024;  // shared memory per CTA for two CTAs per SM
+    int warps_cap = warps_max(pl.MB, pl.CG);
+    bool split = false;
+    if ((flags & MR_GEMV_PDL) && pl.MB <= 4 && n >= 2 * sms &&
+        (size_t)((n + sms - 1) / sms) * k * 2 + (size_t)pl.MB * k * 2 > kPdlBudget) {
+        // A weight block too large for two CTAs per SM (the 31 MB sweep
+        // weight): two CTAs per SM each take half of it through a ring within
+        // the co-residency budget, so that when one exits the next call's CTA
+        // starts streaming in its place (3-4% faster at m <= 4; with 8 or 16
+        // rows A leaves too little room for the ring, and one CTA per SM with
+        // all of the shared memory is faster).
+        pl.G = std::min(2 * sms, n);
+        warps_cap = 8;
+        split = true;
+    }
     const int ng_max = ng_max_of(n, pl.G, pl.CG);
-    const int cwg0 = std::max(1, std::min(ng_max, warps_max(pl.MB, pl.CG) / pl.KW));
+    const int cwg0 = std::max(1, std::min(ng_max, std::max(1, warps_cap / pl.KW)));
     pl.a_bytes = (uint32_t)(((size_t)pl.MB * k * 2 + 127) / 128 * 128);
     pl.slot_bytes = (uint32_t)pl.CG * (uint32_t)k * 2u;
     const size_t red_bytes = red_floats(pl.KW, ng_max, pl.MB, pl.CG) * sizeof(float);
     const size_t topk_bytes = fused ? (size_t)warps_max(pl.MB, pl.CG) * 64 * 8 : 0;
     const size_t fixed = topk_bytes + pl.a_bytes + 24 * (size_t)ng_max + 48 + red_bytes + 64;
-#ifndef MR_GEMV_PDL_BUDGET_KB
-#define MR_GEMV_PDL_BUDGET_KB 110
-#endif
-    const size_t pdl_budget = MR_GEMV_PDL_BUDGET_KB * 1024;
-    const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(pdl_budget, (size_t)optin) : (size_t)optin;
+    const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(kPdlBudget, (size_t)optin) : (size_t)optin;
     auto slots_for = [&](size_t b) -> int {
         if (b <= fixed) return 0;
         return (int)std::min<size_t>((size_t)ng_max, (b - fixed) / pl.slot_bytes);
@@ -661,7 +672,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     int s_max = slots_for(budget);
     if (s_max < 1) s_max = slots_for((size_t)optin);
     if (s_max < 1) return MR_ERR_UNSUPPORTED;
-    if (s_max < ng_max && budget < (size_t)optin) {
+    if (s_max < ng_max && budget < (size_t)optin && !split) {
         // The block does not fit the co-residency budget, so slots would be
         // refilled (a second DRAM round trip per refill).  Streaming depth
         // matters more than overlapping the next launch: take the full shared
