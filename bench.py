@@ -514,7 +514,11 @@ def gemv_curves(rb, flags, hbm_peak):
                 for i in range(max(1, launches // m)):
                     for r in range(m):
                         mr.mrgemv_bf16(A[r:r + 1], pool[i % len(pool)], C[r:r + 1], flags=flags)
+            def warm(m=m, pool=pool, A=A, C=C, launches=launches):
+                for _ in range(launches):
+                    mr.mrgemv_bf16(A[:m], pool[0], C[:m], flags=flags)
             cases.append(((name, m, "batched"), graph_of(torch, stream, batched), launches, 4))
+            cases.append(((name, m, "warm"), graph_of(torch, stream, warm), launches, 4))
             cases.append(((name, m, "per_row"), graph_of(torch, stream, per_row), max(1, launches // m), 2))
             meta[(name, m)] = gemv_bytes(m, n, k)
             if name == "router":
@@ -541,7 +545,8 @@ def gemv_curves(rb, flags, hbm_peak):
             nbytes = meta[(name, m)]
             row = {"us_per_call": b["min"], "us_per_call_median": b["median"], "us_per_row": b["min"] / m,
                    "GBps": nbytes / (b["min"] * 1e3), "frac_of_measured_hbm": nbytes / (b["min"] * 1e3) / hbm_peak,
-                   "per_row_launch_us_per_row": t[(name, m, "per_row")]["min"] / m}
+                   "per_row_launch_us_per_row": t[(name, m, "per_row")]["min"] / m,
+                   "us_per_call_warm_l2": t[(name, m, "warm")]["min"]}
             if name == "router":
                 row["router_fused_us_per_window"] = t[(name, m, "fused")]["min"]
                 row["router_two_launch_us_per_window"] = t[(name, m, "two_launch")]["min"]
@@ -549,7 +554,7 @@ def gemv_curves(rb, flags, hbm_peak):
         cur["batching_speedup_m1_over_m8"] = cur["1"]["us_per_row"] / cur["8"]["us_per_row"]
         out[name] = cur
     out["method"] = (f"min (and median) over {ROUNDS} interleaved rounds of graph-replayed back-to-back calls; "
-                     "weights rotated over copies > 2x L2")
+                     "weights rotated over copies > 2x L2 (us_per_call_warm_l2: the same weight every call)")
     del cases, keep
     return out
 

@@ -120,29 +120,35 @@ mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t flags, int3
  * router_gemv_topk -- the router in one launch: the multi-row GEMV of
  * mrgemv_bf16 followed by the per-row top-k of router_topk.  The two steps of
  * Strata PR #109 ("What", router bullet: one multi-row GEMV plus one multi-row
- * top-10 launch) are fused: every CTA takes an atomic ticket in the workspace
- * once its logits are stored, the last one advances a generation word there,
- * and CTA r (one warp per row) then selects the top-k of row r.  idx / val
- * are bitwise the outputs of mrgemv_bf16 then router_topk on the same inputs.
+ * top-10 launch) are fused: every logit is also stored as a 64-bit word
+ * (a ready flag and the logit's bits) in the workspace's tag array, and CTA r
+ * (one warp per row) polls row r's words until all carry the flag, selects
+ * its top-k and zeroes the words again.  No counter, fence or grid-wide
+ * barrier is involved.  idx / val are bitwise the outputs of mrgemv_bf16 then
+ * router_topk on the same inputs.
  *
  * A, Wt, m, n, k, lda, ldw, flags : as mrgemv_bf16_ex.
  * logits : NULL, or m rows of n fp32 (row stride ldl >= n) that receive the
  *          GEMV output.  When NULL the logits live in the workspace.
  * topk, idx, val, ldo : as router_topk (val may be NULL).
  * workspace : device memory, 256-byte aligned, of at least
- *          router_gemv_topk_workspace_bytes(m, n, logits != NULL) bytes.
- *          Its first MR_ROUTER_TICKET_BYTES must be zero before the first
- *          call; every completed call leaves the ticket counter zero again
- *          (and advances the generation word beside it).  Calls that may
- *          run at the same time (other streams) need separate workspaces.
+ *          router_gemv_topk_workspace_bytes(m, n, logits != NULL) bytes:
+ *          a 256-byte head block (MR_ROUTER_TICKET_BYTES, reserved), the tag
+ *          array of m * n 64-bit words, and -- when logits is NULL -- room
+ *          for the two-launch form's logits in its last m * n * 4 bytes.
+ *          Zero it before the first call: every completed fused call leaves
+ *          the tag array zero again (after a device error, zero it again).
+ *          Calls that share a workspace must pass the same workspace_bytes,
+ *          at least the size for the largest m * n among them.  Calls that
+ *          may run at the same time (other streams) need separate workspaces.
  */
 #define MR_ROUTER_TICKET_BYTES 256u
 /*
  * MR_ROUTER_TWO_LAUNCH (flag of router_gemv_topk / _noalloc): run the window
  * as the GEMV kernel followed by the router_topk kernel (programmatic
  * dependent launch) instead of one fused launch: the same outputs, bit for
- * bit, from one call.  The logits go to `logits`, or to the workspace past
- * its ticket block; the ticket block is not used.
+ * bit, from one call.  The logits go to `logits`, or to the last m * n * 4
+ * bytes of the workspace (rounded down to 256); the tag array is not used.
  */
 #define MR_ROUTER_TWO_LAUNCH 0x4u
 mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt, int64_t ldw,
@@ -162,16 +168,17 @@ size_t router_gemv_topk_workspace_bytes(int32_t m, int32_t n, int32_t logits_pro
  * counterpart: this is a convenience of this library.
  *
  * Arguments and outputs are those of router_gemv_topk.  The scratch it needs
- * (the ticket block, and the logits when `logits` is NULL) is a fixed 256 KiB
- * device array inside the library, held by every GPU that loads the library
- * until the process exits.  With logits == NULL, m * n may not exceed
- * router_gemv_topk_noalloc_max_logits() (65472 values, e.g. 16 x 4092);
- * larger sizes are rejected with MR_ERR_UNSUPPORTED before anything runs.
+ * (the workspace layout of router_gemv_topk) is a fixed 256 KiB device array
+ * inside the library, held by every GPU that loads the library until the
+ * process exits.  With logits == NULL, m * n may not exceed
+ * router_gemv_topk_noalloc_max_logits() (21824 values, e.g. 16 x 1364);
+ * sizes whose workspace does not fit are rejected with MR_ERR_UNSUPPORTED
+ * before anything runs.
  * The call allocates nothing: its first call on a device looks up the array's
  * device address (cudaGetSymbolAddress) with that device current, so make
- * that first call before any stream capture.  Each call clears the ticket on
- * `stream` (cudaMemsetAsync; not with MR_ROUTER_TWO_LAUNCH, which uses no
- * ticket) and then launches.  Every call shares the one
+ * that first call before any stream capture.  Each fused call clears the tag
+ * array on `stream` (cudaMemsetAsync of m * n * 8 bytes; not with
+ * MR_ROUTER_TWO_LAUNCH, which uses no tags) and then launches.  Every call shares the one
  * array, so calls that overlap on the GPU (other streams, or overlapping
  * launches) race and must not be issued.
  */

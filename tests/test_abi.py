@@ -149,10 +149,15 @@ def test_fused_router_validation(kw, code):
 
 
 def test_fused_router_workspace_bytes():
-    assert mr.router_gemv_topk_workspace_bytes(4, 512, True) == 256
-    assert mr.router_gemv_topk_workspace_bytes(4, 512, False) == 256 + 4 * 512 * 4
+    # head block, m x n tagged words, then (no logits passed) m x n fp32; each rounded up to 256 bytes
+    assert mr.router_gemv_topk_workspace_bytes(4, 512, True) == 256 + 4 * 512 * 8
+    assert mr.router_gemv_topk_workspace_bytes(4, 512, False) == 256 + 4 * 512 * 12
+    assert mr.router_gemv_topk_workspace_bytes(1, 3, True) == 256 + 256
+    assert mr.router_gemv_topk_workspace_bytes(1, 3, False) == 256 + 256 + 256
     assert mr.router_gemv_topk_workspace_bytes(0, 512, False) == 0
-    assert fused(logits=P(1024), wsb=256) == mr.MR_ERR_CUDA  # valid; no device here
+    need = mr.router_gemv_topk_workspace_bytes(4, 512, True)
+    assert fused(logits=P(1024), wsb=need) == mr.MR_ERR_CUDA  # valid; no device here
+    assert fused(logits=P(1024), wsb=need - 1) == mr.MR_ERR_INVALID_ARG
 
 
 def test_grouped_validation():

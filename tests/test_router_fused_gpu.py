@@ -1,5 +1,6 @@
 """router_gemv_topk (GEMV + top-k in one launch) against the two-launch path:
-logits, indices and values bitwise equal; the ticket returns to zero."""
+logits, indices and values bitwise equal; the workspace's tag array is all
+zero again after every call."""
 import numpy as np
 import pytest
 
@@ -22,6 +23,11 @@ def _gpu():
 def workspace(m, n, with_logits):
     nbytes = mr.router_gemv_topk_workspace_bytes(m, n, with_logits)
     return torch.zeros((nbytes + 3) // 4, dtype=torch.int32, device="cuda")
+
+
+def tags_are_zero(ws, m, n) -> bool:
+    """The m x n tagged words after the 256-byte head block."""
+    return not host(ws)[64:64 + 2 * m * n].any()
 
 
 def two_launch(A, W, m, n, topk):
@@ -48,8 +54,7 @@ def test_fused_matches_two_launches(m, with_logits):
     assert np.array_equal(host(val).view(np.uint32), v_ref.view(np.uint32))
     if with_logits:
         assert np.array_equal(host(logits).view(np.uint32), c_ref.view(np.uint32))
-    assert int(host(ws)[0]) == 0, "ticket not returned to zero"
-    assert int(host(ws)[16]) == 1, "one call advances the generation word once"
+    assert tags_are_zero(ws, m, 512), "the selecting warps zero the tagged words"
     ri, _ = oracle.topk(c_ref, 10)
     assert np.array_equal(host(idx), ri)
 
@@ -67,6 +72,7 @@ def test_other_shapes(m, n, k, topk):
     mr.router_gemv_topk(A, W, topk, idx, val, workspace=ws)
     assert np.array_equal(host(idx), i_ref)
     assert np.array_equal(host(val).view(np.uint32), v_ref.view(np.uint32))
+    assert tags_are_zero(ws, m, n)
     c64, s64 = oracle.matmul(a, "bf16", w, "bf16")
     ok, worst, _ = oracle.check_matmul(c_ref, c64, s64)
     assert ok, worst
@@ -103,7 +109,26 @@ def test_many_calls_graph_and_pdl_reuse_one_workspace():
     torch.cuda.synchronize()
     for (c, ir, vr), (i, v) in zip(refs, outs):
         assert np.array_equal(host(i), ir)
-    assert int(host(ws)[0]) == 0
+    assert tags_are_zero(ws, 16, 512)
+
+
+def test_fused_and_two_launch_calls_of_any_m_share_one_workspace():
+    """The two-launch form keeps its logits at the end of the workspace, clear
+    of the tag array of any call the workspace was sized for."""
+    ws = workspace(16, 512, False)
+    ws.fill_(0)
+    seq = [(16, 0), (1, mr.MR_ROUTER_TWO_LAUNCH), (16, 0), (4, mr.MR_ROUTER_TWO_LAUNCH), (8, 0), (16, 0)]
+    for i, (m, form) in enumerate(seq):
+        a = synth.normal_bits(1300 + i, (m, 2560), "bf16", 1.0)
+        w = synth.normal_bits(1350 + i, (512, 2560), "bf16", 0.02)
+        A, W = dev_bits(a), dev_bits(w)
+        _, ir, vr = two_launch(A, W, m, 512, 10)
+        idx = torch.empty((m, 10), dtype=torch.int32, device="cuda")
+        val = torch.empty((m, 10), dtype=torch.float32, device="cuda")
+        mr.router_gemv_topk(A, W, 10, idx, val, workspace=ws, flags=mr.MR_GEMV_PDL | form)
+        assert np.array_equal(host(idx), ir), (i, m, form)
+        assert np.array_equal(host(val).view(np.uint32), vr.view(np.uint32)), (i, m, form)
+        assert tags_are_zero(ws, 16, 512), (i, m, form)
 
 
 @pytest.mark.parametrize("m", [1, 5, 16])
@@ -114,7 +139,7 @@ def test_two_launch_flag_matches_fused_and_separate_calls(m, with_logits):
     A, W = dev_bits(a), dev_bits(w)
     c_ref, i_ref, v_ref = two_launch(A, W, m, 512, 10)
     ws = workspace(m, 512, with_logits)
-    ws.fill_(-1)   # the ticket block is not used by this form
+    ws.fill_(-1)   # neither the head block nor the tag array is used by this form
     idx = torch.full((m, 10), -1, dtype=torch.int32, device="cuda")
     val = torch.full((m, 10), float("nan"), dtype=torch.float32, device="cuda")
     logits = torch.empty((m, 512), dtype=torch.float32, device="cuda") if with_logits else None
@@ -125,7 +150,8 @@ def test_two_launch_flag_matches_fused_and_separate_calls(m, with_logits):
     if with_logits:
         assert np.array_equal(host(logits).view(np.uint32), c_ref.view(np.uint32))
     else:
-        got = host(ws)[64:64 + m * 512].view(np.float32).reshape(m, 512)
+        off = (ws.numel() * 4 - m * 512 * 4) // 256 * 256 // 4   # the last m * n * 4 bytes
+        got = host(ws)[off:off + m * 512].view(np.float32).reshape(m, 512)
         assert np.array_equal(got.view(np.uint32), c_ref.view(np.uint32))
     with pytest.raises(mr.MrError):
         mr.router_gemv_topk(A, W, 10, idx, val, workspace=ws, flags=mr.MR_GEMV_SIGMOID)

@@ -228,9 +228,10 @@ def router_gemv_topk_workspace_bytes(m: int, n: int, logits_provided: bool) -> i
 
 def router_gemv_topk(A, Wt, topk: int, idx, val=None, logits=None, workspace=None, stream=None,
                      flags: int = 0) -> None:
-    """GEMV + per-row top-k in one launch.  ``workspace``: a CUDA tensor of at
-    least router_gemv_topk_workspace_bytes(...) bytes whose first 256 bytes are
-    zero before the first call (each call leaves them zero)."""
+    """GEMV + per-row top-k in one launch (or, with MR_ROUTER_TWO_LAUNCH, the
+    GEMV kernel then the top-k kernel).  ``workspace``: a zeroed CUDA tensor
+    of at least router_gemv_topk_workspace_bytes(...) bytes (each fused call
+    leaves its tag array zero again)."""
     m, k, lda = _rows(A, "A")
     n, kw, ldw = _rows(Wt, "Wt")
     if kw != k:

@@ -62,9 +62,14 @@ constexpr int kWarpsMax = 16;
 __host__ __device__ constexpr int warps_max(int, int) { return kWarpsMax; }
 __host__ __device__ constexpr int q_unroll(int MB, int) { return MB >= 8 ? MR_GEMV_UNROLL_LARGE : MR_GEMV_UNROLL_SMALL; }
 constexpr int kMaxRows = 16;
-// Word of the fused router's ticket block that counts completed calls (the
-// counter itself is word 0; 64 bytes apart).
-constexpr int kGenerationWord = 16;
+// Fused router: each logit is also stored as one 64-bit word, the flag
+// kTagReady in the high half and the logit's bits in the low half, in a tag
+// array of the workspace that is all zero between calls.  A 64-bit store is
+// single-copy atomic, so a word that carries the flag carries its logit too.
+constexpr uint32_t kTagReady = 1u;
+#ifndef MR_FUSED_P
+#define MR_FUSED_P 16   // logits per lane per segment in the fused selection
+#endif
 
 struct Params {
     const uint16_t *A;
@@ -86,7 +91,7 @@ struct Params {
     int32_t *idx;
     float *val;
     int64_t ldo;
-    uint32_t *ticket;     // CTAs that finished their columns (0 between calls)
+    uint64_t *tags;       // m x n tagged logits, row stride n (zero between calls)
 };
 
 // k-slice split: a function of k alone (never of m), so the reduction tree of
@@ -115,6 +120,61 @@ __host__ __device__ inline int k_warps(int k) {
 // expf and an IEEE divide.
 __device__ __forceinline__ float gate_out(const Params &p, float c) {
     return p.sigmoid ? 1.0f / (1.0f + expf(-c)) : c;
+}
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *a) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a) : "memory");
+    return v;
+}
+
+// Output of logit (r, col): to C, and in the fused router (where C may be
+// null) also as a tagged word with a GPU-scope relaxed store.
+template <bool FUSED>
+__device__ __forceinline__ void store_logit(const Params &p, int r, int col, float v) {
+    if (!FUSED || p.C) p.C[(int64_t)r * p.ldc + col] = v;
+    if constexpr (FUSED)
+        asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p.tags + (int64_t)r * p.n + col),
+                     "l"(((uint64_t)kTagReady << 32) | __float_as_uint(v))
+                     : "memory");
+}
+
+// Top-k of one row of tagged logits, taken by one warp in segments of 32 * P
+// words: each segment's words are re-read until all carry the flag (bounded
+// by kWaitLimitNs; false if it runs out), then keyed and merged like
+// router_topk's rows.  `out`: lane t holds the rank-t key.
+template <int P>
+__device__ __forceinline__ bool tagged_topk(const uint64_t *row, int n, int K, int lane, uint64_t *scratch,
+                                            uint64_t &out) {
+    const uint64_t t0 = globaltimer_ns();
+    uint64_t run = 0ull;
+    for (int base = 0; base < n; base += 32 * P) {
+        uint64_t w[P];
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            const int j = base + lane + 32 * i;
+            w[i] = j < n ? ld_relaxed_u64(row + j) : ((uint64_t)kTagReady << 32);
+        }
+        for (int spin = 0;; ++spin) {
+            bool ready = true;
+#pragma unroll
+            for (int i = 0; i < P; ++i) ready = ready && (uint32_t)(w[i] >> 32) == kTagReady;
+            if (__all_sync(0xffffffffu, ready)) break;
+            if ((spin & 15) == 15 && __any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitLimitNs)) return false;
+#pragma unroll
+            for (int i = 0; i < P; ++i)
+                if ((uint32_t)(w[i] >> 32) != kTagReady) w[i] = ld_relaxed_u64(row + base + lane + 32 * i);
+        }
+        uint64_t keys[P];
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            const int j = base + lane + 32 * i;
+            keys[i] = j < n ? topk::make_key(__uint_as_float((uint32_t)w[i]), (uint32_t)j) : 0ull;
+        }
+        run = topk::warp_topk_merge<P>(keys, run, K, lane, scratch);
+    }
+    out = run;
+    return true;
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -196,13 +256,11 @@ struct Smem {
     uint64_t *empty;      // [S]
     uint64_t *a_full;     // [1] A has landed (A staged by a bulk copy)
     uint64_t *parts_done; // [1] every warp has written its k-slice partials
-    uint64_t *cta_done;   // [1] every warp's logits are stored (fused router)
-    uint32_t *gen0;       // [2] the workspace's generation word before this call
     float *red;           // [groups][KW][MB x CG] k-slice partials (KW > 1)
 };
 
 // One column group: NC (power of two) columns of this warp's k-slice.
-template <int MB, int NC, int CGMAX>
+template <int MB, int NC, int CGMAX, bool FUSED>
 __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g, int ncol,
                                          int col0, int slice, int lane, int q_begin, int q_end,
                                          int chunk_groups) {
@@ -327,22 +385,22 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
             for (int i = 0; i < PL; ++i) {
                 const int idx = base + i;
                 const int r = idx / NC, j = idx % NC;
-                if (r < p.m && j < ncol) p.C[(int64_t)r * p.ldc + col0 + j] = gate_out(p, v[i]);
+                if (r < p.m && j < ncol) store_logit<FUSED>(p, r, col0 + j, gate_out(p, v[i]));
             }
         }
     }
     return true;
 }
 
-template <int MB, int NC, int CGMAX>
+template <int MB, int NC, int CGMAX, bool FUSED>
 __device__ __forceinline__ bool run_group(const Params &p, const Smem &sm, int g, int ncol,
                                           int col0, int slice, int lane, int q_begin, int q_end,
                                           int chunk_groups) {
     if constexpr (NC > 1) {
         if (ncol <= NC / 2)
-            return run_group<MB, NC / 2, CGMAX>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups);
+            return run_group<MB, NC / 2, CGMAX, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups);
     }
-    return do_group<MB, NC, CGMAX>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups);
+    return do_group<MB, NC, CGMAX, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups);
 }
 
 template <int MB, int CG, bool FUSED>
@@ -366,10 +424,8 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     sm.chunk_full = reinterpret_cast<uint64_t *>(sm.ring + (size_t)p.S * p.slot_bytes);
     sm.full = sm.chunk_full + p.S;
     sm.empty = sm.full + p.S;
-    uint64_t *misc = sm.empty + p.S;  // 6 words: barriers and the last-CTA flag
+    uint64_t *misc = sm.empty + p.S;  // 6 words: two barriers and spare words
     sm.a_full = misc;
-    sm.cta_done = misc + 1;
-    sm.gen0 = reinterpret_cast<uint32_t *>(misc + 3);
     sm.parts_done = misc + 5;
     sm.red = reinterpret_cast<float *>(misc + 6);
 
@@ -418,7 +474,6 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
         }
         mbar_init(smem_u32(sm.a_full), 1);
         mbar_init(smem_u32(sm.parts_done), (uint32_t)(blockDim.x / 32));
-        if constexpr (FUSED) mbar_init(smem_u32(sm.cta_done), (uint32_t)(blockDim.x / 32));
         fence_mbar_init();
         // The whole first pass of the ring (min(ng, S) groups) is requested
         // now, before the wait for the previous kernel, in chunks of whole
@@ -431,13 +486,6 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     grid_launch_dependents();
     // A may be produced by the previous kernel on the stream.
     grid_dependency_wait();
-    if constexpr (FUSED) {
-        // The generation before this call: read after the previous kernel
-        // (possibly a fused call on the same workspace) has completed.
-        if (tid == 0)
-            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(*sm.gen0) : "l"(p.ticket + kGenerationWord)
-                         : "memory");
-    }
 
     // Stage A (bf16) in shared memory with one bulk copy (per row if strided);
     // rows m..MB-1 are zero.  Under programmatic dependent launch the weight
@@ -473,7 +521,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     for (int g = cw; g < ng && !failed; g += p.CWG) {
         const int col0 = c_begin + g * CG;
         const int ncol = min(CG, c_end - col0);
-        if (!run_group<MB, CG, CG>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups)) {
+        if (!run_group<MB, CG, CG, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups)) {
             failed = true;
             break;
         }
@@ -507,62 +555,44 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
                 const float *src = sm.red + (size_t)g * p.KW * VCG + rem;
                 float acc = src[0];
                 for (int sl = 1; sl < p.KW; ++sl) acc = __fadd_rn(acc, src[(size_t)sl * VCG]);
-                p.C[(int64_t)r * p.ldc + col] = gate_out(p, acc);
+                store_logit<FUSED>(p, r, col, gate_out(p, acc));
             }
         }
     }
 
     if constexpr (FUSED) {
-        // Router top-k in the same launch.  Every warp releases its logits
-        // (cta_done); thread 0 then takes a ticket (acq_rel at GPU scope).
-        // The CTA that draws the last ticket resets the counter and advances
-        // the workspace's generation word with a release store.  CTA b
-        // selects rows b, b + G, ... with one warp per row: lane 0 waits,
-        // bounded, for the generation to move past the value read after the
-        // grid-dependency wait, and the warp then reads the row from L2 (every
-        // CTA's stores are ordered before the last ticket, and that before
-        // the generation) and selects.  The m rows are selected in parallel
-        // on m SMs.  Every warp arrives even after a failed wait, so thread
-        // 0's wait ends.
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(sm.cta_done));
-        uint32_t *gen = p.ticket + kGenerationWord;
-        if (warp == 0 && mbar_wait_bounded(smem_u32(sm.cta_done), 0u, MR_DEVERR_GEMV_TIMEOUT) && lane == 0) {
-            asm volatile("fence.acq_rel.gpu;" ::: "memory");
-            uint32_t t;
-            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.ticket) : "memory");
-            if (t == (uint32_t)p.G - 1u) {
-                *p.ticket = 0u;  // the counter starts at zero for the next call
-                asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(gen), "r"(*sm.gen0 + 1u) : "memory");
-            }
-        }
+        // Router top-k in the same launch, with no fence, counter or barrier
+        // across CTAs: CTA b selects rows b, b + G, ... with one warp per row.
+        // The warp polls the row's tagged words (GPU-scope relaxed loads,
+        // bounded) until every one carries the flag, which it does once the
+        // CTA that owns its column has stored it; it then selects the top-k
+        // under the router's total order, writes idx / val, and zeroes the
+        // row's words for the next call (the next kernel on the stream starts
+        // storing only after this one has completed).  Only the <= m CTAs
+        // that select wait, each after storing its own columns, so the other
+        // CTAs always run to completion.
         const int nwarps = blockDim.x >> 5;
-        int r = (int)blockIdx.x + warp * p.G;
-        if (r >= p.m) return;
-        uint32_t ok = 1u;
-        if (lane == 0) {
-            const uint32_t g0 = *sm.gen0;
-            const uint64_t t0 = globaltimer_ns();
-            uint32_t g;
-            for (int spin = 0;; ++spin) {
-                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(gen) : "memory");
-                if (g != g0) break;
-                if ((spin & 63) == 63 && globaltimer_ns() - t0 > kWaitLimitNs) {
-                    record_error(MR_DEVERR_GEMV_TIMEOUT);
-                    ok = 0u;
-                    break;
+        // 64 keys of 16-byte aligned scratch per warp after the k-slice partials.
+        const uintptr_t tk0 = reinterpret_cast<uintptr_t>(sm.red + red_floats(p.KW, ng_max_of(p.n, p.G, CG), MB, CG));
+        uint64_t *tk = reinterpret_cast<uint64_t *>((tk0 + 15u) & ~(uintptr_t)15u) + warp * 64;
+        for (int r = (int)blockIdx.x + warp * p.G; r < p.m; r += nwarps * p.G) {
+            uint64_t *row = p.tags + (int64_t)r * p.n;
+            uint64_t best = 0ull;
+            if (!tagged_topk<MR_FUSED_P>(row, p.n, p.topk, lane, tk, best)) {
+                if (lane == 0) record_error(MR_DEVERR_GEMV_TIMEOUT);
+                return;
+            }
+            if (lane < p.topk) {
+                const uint32_t j = topk::key_index(best);
+                p.idx[(int64_t)r * p.ldo + lane] = (int32_t)j;
+                if (p.val) {
+                    bool exact;
+                    const float v = topk::key_value(best, exact);
+                    p.val[(int64_t)r * p.ldo + lane] = exact ? v : __uint_as_float((uint32_t)ld_relaxed_u64(row + j));
                 }
             }
-        }
-        if (__shfl_sync(0xffffffffu, ok, 0) == 0u) return;
-        uint64_t *tk = reinterpret_cast<uint64_t *>(sm.red + red_floats(p.KW, ng_max_of(p.n, p.G, CG), MB, CG)) + warp * 64;
-        for (; r < p.m; r += nwarps * p.G) {
-            const float *x = p.C + (int64_t)r * p.ldc;
-            const uint64_t best = topk::warp_topk_fast<16, true>(x, p.n, p.topk, lane, 0, 1, 0ull, tk);
-            if (lane < p.topk) {
-                p.idx[(int64_t)r * p.ldo + lane] = (int32_t)topk::key_index(best);
-                if (p.val) p.val[(int64_t)r * p.ldo + lane] = topk::selected_value<true>(best, x);
-            }
+            __syncwarp();
+            for (int j = lane; j < p.n; j += 32) row[j] = 0ull;
         }
     }
 }
@@ -662,7 +692,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     pl.a_bytes = (uint32_t)(((size_t)pl.MB * k * 2 + 127) / 128 * 128);
     pl.slot_bytes = (uint32_t)pl.CG * (uint32_t)k * 2u;
     const size_t red_bytes = red_floats(pl.KW, ng_max, pl.MB, pl.CG) * sizeof(float);
-    const size_t topk_bytes = fused ? (size_t)warps_max(pl.MB, pl.CG) * 64 * 8 : 0;
+    const size_t topk_bytes = fused ? (size_t)warps_max(pl.MB, pl.CG) * 64 * 8 + 16 : 0;
     const size_t fixed = topk_bytes + pl.a_bytes + 24 * (size_t)ng_max + 48 + red_bytes + 64;
     const size_t budget = (flags & MR_GEMV_PDL) ? std::min<size_t>(kPdlBudget, (size_t)optin) : (size_t)optin;
     auto slots_for = [&](size_t b) -> int {
@@ -721,7 +751,7 @@ struct FusedArgs {
     int32_t *idx;
     float *val;
     int64_t ldo;
-    uint32_t *ticket;
+    uint64_t *tags;
 };
 
 // Validate and plan a launch without touching the device or any stream:
@@ -729,7 +759,7 @@ struct FusedArgs {
 // adds the router top-k of every row.
 mr_status prepare(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *C, int64_t ldc, int32_t m,
                   int32_t n, int32_t k, uint32_t flags, const FusedArgs *fused, Params &p, Plan &pl) {
-    if (!A || !Wt || !C) return MR_ERR_INVALID_ARG;
+    if (!A || !Wt || (!C && !fused)) return MR_ERR_INVALID_ARG;
     if (m < 1 || n < 1 || k < 1) return MR_ERR_INVALID_ARG;
     if (lda < k || ldw < k || ldc < n) return MR_ERR_INVALID_ARG;
     if (flags & ~(MR_GEMV_PDL | MR_GEMV_SIGMOID)) return MR_ERR_INVALID_ARG;
@@ -766,7 +796,7 @@ mr_status prepare(const void *A, int64_t lda, const void *Wt, int64_t ldw, float
         p.idx = fused->idx;
         p.val = fused->val;
         p.ldo = fused->ldo;
-        p.ticket = fused->ticket;
+        p.tags = fused->tags;
     }
     return MR_OK;
 }
@@ -806,7 +836,8 @@ mr_status launch(const void *A, int64_t lda, const void *Wt, int64_t ldw, float 
 // GEMV's; nothing is enqueued.  On success p and pl describe the launch.
 mr_status prepare_router(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *logits, int64_t ldl,
                          int32_t m, int32_t n, int32_t k, int32_t topk, int32_t *idx, float *val, int64_t ldo,
-                         void *workspace, size_t workspace_bytes, uint32_t flags, Params &p, Plan &pl);
+                         void *workspace, size_t workspace_bytes, uint32_t flags, bool two_launch, Params &p,
+                         Plan &pl);
 
 }  // namespace gemv
 }  // namespace mr
@@ -817,9 +848,19 @@ extern "C" mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, 
     return mr::gemv::launch(A, lda, Wt, ldw, C, ldc, m, n, k, flags, stream, nullptr);
 }
 
+// Workspace layout: a reserved head block, the tag array (m x n words) at
+// offset MR_ROUTER_TICKET_BYTES, and -- when the caller passes no logits --
+// the two-launch form's fp32 logits in the last m * n * 4 bytes (rounded down
+// to 256), so that calls of any m * n up to the size the workspace was made
+// for never put logits where another call's tags are.
+namespace {
+size_t align256(size_t b) { return (b + 255u) & ~(size_t)255u; }
+}  // namespace
+
 extern "C" size_t router_gemv_topk_workspace_bytes(int32_t m, int32_t n, int32_t logits_provided) {
     if (m < 1 || n < 1) return 0;
-    return MR_ROUTER_TICKET_BYTES + (logits_provided ? 0 : (size_t)m * (size_t)n * sizeof(float));
+    const size_t mn = (size_t)m * (size_t)n;
+    return MR_ROUTER_TICKET_BYTES + align256(mn * 8u) + (logits_provided ? 0 : align256(mn * sizeof(float)));
 }
 
 namespace mr {
@@ -827,7 +868,8 @@ namespace gemv {
 
 mr_status prepare_router(const void *A, int64_t lda, const void *Wt, int64_t ldw, float *logits, int64_t ldl,
                          int32_t m, int32_t n, int32_t k, int32_t topk, int32_t *idx, float *val, int64_t ldo,
-                         void *workspace, size_t workspace_bytes, uint32_t flags, Params &p, Plan &pl) {
+                         void *workspace, size_t workspace_bytes, uint32_t flags, bool two_launch, Params &p,
+                         Plan &pl) {
     if (!idx || !workspace) return MR_ERR_INVALID_ARG;
     if (m < 1 || n < 1 || topk < 1 || topk > n || ldo < topk) return MR_ERR_INVALID_ARG;
     if (topk > 32) return MR_ERR_UNSUPPORTED;
@@ -836,11 +878,16 @@ mr_status prepare_router(const void *A, int64_t lda, const void *Wt, int64_t ldw
     float *C = logits;
     int64_t ldc = ldl;
     if (!C) {
-        C = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + MR_ROUTER_TICKET_BYTES);
+        const size_t off = (workspace_bytes - (size_t)m * (size_t)n * sizeof(float)) & ~(size_t)255u;
+        C = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + off);
         ldc = n;
     }
-    const FusedArgs fa = {topk, idx, val, ldo, static_cast<uint32_t *>(workspace)};
-    return prepare(A, lda, Wt, ldw, C, ldc, m, n, k, flags, &fa, p, pl);
+    uint64_t *tags = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(workspace) + MR_ROUTER_TICKET_BYTES);
+    const FusedArgs fa = {topk, idx, val, ldo, tags};
+    const mr_status st = prepare(A, lda, Wt, ldw, C, ldc, m, n, k, flags, &fa, p, pl);
+    // The fused form stores the workspace logits only as tagged words.
+    if (st == MR_OK && !logits && !two_launch) p.C = nullptr;
+    return st;
 }
 
 }  // namespace gemv
@@ -870,7 +917,8 @@ extern "C" mr_status router_gemv_topk(const void *A, int64_t lda, const void *Wt
     mr::gemv::Params p;
     mr::gemv::Plan pl;
     const mr_status st = mr::gemv::prepare_router(A, lda, Wt, ldw, logits, ldl, m, n, k, topk, idx, val, ldo,
-                                                  workspace, workspace_bytes, flags & ~MR_ROUTER_TWO_LAUNCH, p, pl);
+                                                  workspace, workspace_bytes, flags & ~MR_ROUTER_TWO_LAUNCH,
+                                                  (flags & MR_ROUTER_TWO_LAUNCH) != 0, p, pl);
     if (st != MR_OK) return st;
     return mr::gemv::launch_router(p, pl, flags, stream);
 }
@@ -918,8 +966,10 @@ mr_status noalloc_scratch(void **out) {
 }  // namespace gemv
 }  // namespace mr
 
+// With no logits passed, m * n values take 12 bytes each (a tagged word and
+// an fp32 logit); a multiple of 64 keeps both arrays whole 256-byte blocks.
 extern "C" size_t router_gemv_topk_noalloc_max_logits(void) {
-    return (mr::gemv::kNoAllocScratchBytes - MR_ROUTER_TICKET_BYTES) / sizeof(float);
+    return (mr::gemv::kNoAllocScratchBytes - MR_ROUTER_TICKET_BYTES) / 12u / 64u * 64u;
 }
 
 extern "C" mr_status router_gemv_topk_noalloc(const void *A, int64_t lda, const void *Wt, int64_t ldw,
@@ -927,7 +977,8 @@ extern "C" mr_status router_gemv_topk_noalloc(const void *A, int64_t lda, const 
                                               int32_t topk, int32_t *idx, float *val, int64_t ldo, uint32_t flags,
                                               void *stream) {
     if (m < 1 || n < 1) return MR_ERR_INVALID_ARG;
-    if (!logits && (size_t)m * (size_t)n > router_gemv_topk_noalloc_max_logits()) return MR_ERR_UNSUPPORTED;
+    if (router_gemv_topk_workspace_bytes(m, n, logits != nullptr) > mr::gemv::kNoAllocScratchBytes)
+        return MR_ERR_UNSUPPORTED;
     void *scratch = nullptr;
     mr_status st = mr::gemv::noalloc_scratch(&scratch);
     if (st != MR_OK) return st;
@@ -935,12 +986,14 @@ extern "C" mr_status router_gemv_topk_noalloc(const void *A, int64_t lda, const 
     if (flags & ~(MR_GEMV_PDL | MR_ROUTER_TWO_LAUNCH)) return MR_ERR_INVALID_ARG;
     mr::gemv::Params p;
     mr::gemv::Plan pl;
+    const bool two_launch = (flags & MR_ROUTER_TWO_LAUNCH) != 0;
     st = mr::gemv::prepare_router(A, lda, Wt, ldw, logits, ldl, m, n, k, topk, idx, val, ldo, scratch,
-                                  mr::gemv::kNoAllocScratchBytes, flags & ~MR_ROUTER_TWO_LAUNCH, p, pl);
+                                  mr::gemv::kNoAllocScratchBytes, flags & ~MR_ROUTER_TWO_LAUNCH, two_launch, p, pl);
     if (st != MR_OK) return st;
-    // The array keeps whatever the last call left; the ticket must start at zero.
-    if (!(flags & MR_ROUTER_TWO_LAUNCH) &&
-        cudaMemsetAsync(scratch, 0, MR_ROUTER_TICKET_BYTES, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    // The array keeps whatever the last call left (a call that failed on the
+    // device may leave tagged words behind); the tags must start at zero.
+    if (!two_launch && cudaMemsetAsync(p.tags, 0, (size_t)m * (size_t)n * 8u, static_cast<cudaStream_t>(stream)) !=
+                           cudaSuccess)
         return MR_ERR_CUDA;
     return mr::gemv::launch_router(p, pl, flags, stream);
 }

@@ -14,16 +14,17 @@ namespace topk {
 // is 0xFFFFFFFF - index, so the lower index of two equal values has the
 // larger key.  0 is never a key (it would need index 0xFFFFFFFF) and marks an
 // empty entry.
+__device__ __forceinline__ uint32_t order_word(float v) {
+    const uint32_t b = __float_as_uint(v);
+    // b ^ 0x80000000 for a clear sign bit (b | 0x80000000), ~b for a set one
+    uint32_t hi = b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+    hi = (b == 0x80000000u) ? 0x80000000u : hi;  // -0.0 onto +0.0
+    hi = (v != v) ? 0xFFFFFFFFu : hi;            // every NaN to the maximum
+    return hi;
+}
+
 __device__ __forceinline__ uint64_t make_key(float v, uint32_t idx) {
-    uint32_t b = __float_as_uint(v);
-    uint32_t hi;
-    if (v != v) {
-        hi = 0xFFFFFFFFu;
-    } else {
-        if ((b & 0x7FFFFFFFu) == 0u) b = 0u;
-        hi = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    }
-    return ((uint64_t)hi << 32) | (uint64_t)(0xFFFFFFFFu - idx);
+    return ((uint64_t)order_word(v) << 32) | (uint64_t)(0xFFFFFFFFu - idx);
 }
 
 __device__ __forceinline__ uint32_t key_index(uint64_t key) { return 0xFFFFFFFFu - (uint32_t)key; }
@@ -88,85 +89,104 @@ __device__ __forceinline__ uint64_t warp_select(uint64_t (&x)[L], int K, int lan
     return mine;
 }
 
-// Running top-K of elements [begin, end) of a row taken by one warp in
-// segments of 32*P elements starting at `begin` and stepping `stride`
-// segments; `run` is the warp's running list (lane t holds rank t).
-template <int P>
-__device__ __forceinline__ uint64_t warp_topk_segments(const float *x, int n, int K, int lane, int seg0,
-                                                       int seg_stride, uint64_t run) {
-    for (int seg = seg0; (int64_t)seg * 32 * P < n; seg += seg_stride) {
-        const int base = seg * 32 * P;
-        uint64_t keys[P + 1];
-#pragma unroll
-        for (int i = 0; i < P; ++i) {
-            const int j = base + lane + 32 * i;
-            keys[i] = j < n ? make_key(x[j], (uint32_t)j) : 0ull;
-        }
-        keys[P] = run;
-        sort_desc(keys);
-        run = warp_select(keys, K, lane);
-    }
-    return run;
-}
-
-// Rank of `key` among the 32 lanes' keys: how many lanes hold a larger key.
-// Keys are unique, so nonzero keys get distinct ranks.
-__device__ __forceinline__ int warp_rank(uint64_t key, int lane) {
-    int r = 0;
-#pragma unroll
-    for (int s = 1; s < 32; ++s) {
-        const uint64_t o = __shfl_sync(0xffffffffu, key, (lane + s) & 31);
-        r += o > key ? 1 : 0;
-    }
-    return r;
+// The heavy-tie fallback of warp_topk_merge: sort each lane's L keys and
+// take K rounds of the warp-wide maximum.  Kept out of line: inlined, its
+// sorting network is scheduled into the common path and slows it by about
+// half although it never runs there.
+template <int L>
+struct KeySet {
+    uint64_t k[L];
+};
+template <int L>
+__device__ __noinline__ uint64_t select_rounds(KeySet<L> all, int K, int lane) {
+    sort_desc(all.k);
+    return warp_select(all.k, K, lane);
 }
 
 // Top-K (K <= 32) of one chunk of up to 32*P keys held P per lane, merged
-// with a running list `run` (lane t holds rank t, 0 = empty).  Fast path:
-// tau = the K-th largest lane maximum (every one of the top K keys is >= tau,
-// because the K lanes with the largest maxima each hold a key >= tau); the
-// keys >= tau are gathered through `scratch` (64 keys of shared memory per
-// warp) and, when there are at most 32, ranked with shuffles in one pass.
-// Otherwise (heavy ties) it falls back to K rounds of warp-wide maximum.
+// with a running list `run` (lane t holds rank t, 0 = empty).  `scratch`:
+// 64 keys of shared memory for this warp, 16-byte aligned.
+//  1. tau = the K-th largest lane maximum of the keys' high words (the
+//     largest value that at least K lanes reach): every one of the top K keys
+//     has a high word >= tau, since the K lanes that reach tau each hold one.
+//     The lane maxima are exchanged through shared memory (broadcast reads),
+//     not shuffles.
+//  2. The keys with a high word >= tau are the candidates; each lane's count
+//     is prefix-summed over the lanes bit by bit (one ballot per bit) and the
+//     candidates are stored to consecutive slots of `scratch`.
+//  3. When there are at most 32, lane t takes candidate t and ranks it by
+//     comparing with all of them (broadcast reads again); the rank-r key is
+//     written to slot 32 + r.  Otherwise (heavy ties) select_rounds.
 // Returns the new running list (lane t holds rank t).
 template <int P>
 __device__ __forceinline__ uint64_t warp_topk_merge(uint64_t (&key)[P], uint64_t run, int K, int lane,
                                                     uint64_t *scratch) {
-    // Lane maximum by a pairwise tree (short dependency chain).
-    uint64_t t[P];
+    static_assert(P + 1 <= 31, "one mask bit per key");
+    uint32_t hi[P + 1], t[P + 1];
 #pragma unroll
-    for (int i = 0; i < P; ++i) t[i] = key[i];
+    for (int i = 0; i < P; ++i) hi[i] = (uint32_t)(key[i] >> 32);
+    hi[P] = (uint32_t)(run >> 32);
 #pragma unroll
-    for (int w = 1; w < P; w <<= 1)
+    for (int i = 0; i <= P; ++i) t[i] = hi[i];
 #pragma unroll
-        for (int i = 0; i + w < P; i += 2 * w) t[i] = t[i + w] > t[i] ? t[i + w] : t[i];
-    const uint64_t mx = t[0] > run ? t[0] : run;
-    const int r0 = warp_rank(mx, lane);
-    const unsigned who = __ballot_sync(0xffffffffu, r0 == K - 1 && mx != 0ull);
-    // Fewer than K nonzero lane maxima: every nonzero key is a candidate.
-    const uint64_t tau = who ? __shfl_sync(0xffffffffu, mx, __ffs(who) - 1) : 1ull;
-    int c = (run >= tau && run != 0ull) ? 1 : 0;
+    for (int w = 1; w < P + 1; w <<= 1)
 #pragma unroll
-    for (int i = 0; i < P; ++i) c += (key[i] >= tau && key[i] != 0ull) ? 1 : 0;
-    int pos = c;  // inclusive prefix sum of the counts over lanes
+        for (int i = 0; i + w < P + 1; i += 2 * w) t[i] = max(t[i], t[i + w]);
+    const uint32_t mx = t[0];
+    uint32_t *s32 = reinterpret_cast<uint32_t *>(scratch);
+    s32[lane] = mx;
+    __syncwarp();
+    int g0 = 0, g1 = 0, g2 = 0, g3 = 0;  // lanes whose maximum is >= this lane's
+    const uint4 *q = reinterpret_cast<const uint4 *>(s32);
 #pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, pos, d);
-        if (lane >= d) pos += o;
+    for (int j = 0; j < 8; ++j) {
+        const uint4 w = q[j];
+        g0 += w.x >= mx ? 1 : 0;
+        g1 += w.y >= mx ? 1 : 0;
+        g2 += w.z >= mx ? 1 : 0;
+        g3 += w.w >= mx ? 1 : 0;
     }
-    const int total = __shfl_sync(0xffffffffu, pos, 31);
-    if (total <= 32) {
-        pos -= c;
-        if (c) {
-            if (run >= tau && run != 0ull) scratch[pos++] = run;
+    const int ge = (g0 + g1) + (g2 + g3);
+    // An empty key has a zero high word and no real key does: tau >= 1.
+    const uint32_t tau = max(__reduce_max_sync(0xffffffffu, ge >= K ? mx : 0u), 1u);
+    uint32_t msk = 0;
 #pragma unroll
-            for (int i = 0; i < P; ++i)
-                if (key[i] >= tau && key[i] != 0ull) scratch[pos++] = key[i];
+    for (int i = 0; i <= P; ++i) msk |= (hi[i] >= tau ? 1u : 0u) << i;
+    const uint32_t c = (uint32_t)__popc(msk);
+    const unsigned below = (1u << lane) - 1u;
+    int pos = 0, total = 0;
+#pragma unroll
+    for (int b = 0; (1 << b) <= P + 1; ++b) {
+        const unsigned bb = __ballot_sync(0xffffffffu, (c >> b) & 1u);
+        pos += __popc(bb & below) << b;
+        total += __popc(bb) << b;
+    }
+    if (total <= 32) {
+        __syncwarp();  // every lane has read the maxima
+        int slot = pos;
+#pragma unroll
+        for (int i = 0; i <= P; ++i) {
+            const uint32_t take = (msk >> i) & 1u;
+            const uint32_t addr = (uint32_t)__cvta_generic_to_shared(scratch + slot);
+            asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q st.shared.u64 [%0], %1;\n\t}" ::"r"(addr),
+                         "l"(i < P ? key[i] : run), "r"(take)
+                         : "memory");
+            slot += (int)take;
         }
         scratch[32 + lane] = 0ull;
         __syncwarp();
         const uint64_t cand = lane < total ? scratch[lane] : 0ull;
-        const int r = warp_rank(cand, lane);
+        int r0 = 0, r1 = 0, r2 = 0, r3 = 0;  // candidates larger than this lane's
+        const ulonglong2 *q2 = reinterpret_cast<const ulonglong2 *>(scratch);
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+            const ulonglong2 a = q2[j], b = q2[j + 1];
+            r0 += (2 * j + 0 < total && a.x > cand) ? 1 : 0;
+            r1 += (2 * j + 1 < total && a.y > cand) ? 1 : 0;
+            r2 += (2 * j + 2 < total && b.x > cand) ? 1 : 0;
+            r3 += (2 * j + 3 < total && b.y > cand) ? 1 : 0;
+        }
+        const int r = (r0 + r1) + (r2 + r3);
         __syncwarp();
         if (cand != 0ull && r < K) scratch[32 + r] = cand;
         __syncwarp();
@@ -174,27 +194,29 @@ __device__ __forceinline__ uint64_t warp_topk_merge(uint64_t (&key)[P], uint64_t
         __syncwarp();
         return out;
     }
-    // Slow path: sort each lane's keys and take K rounds of the warp maximum.
-    uint64_t all[P + 1];
+    KeySet<P + 1> all;
 #pragma unroll
-    for (int i = 0; i < P; ++i) all[i] = key[i];
-    all[P] = run;
-    sort_desc(all);
-    return warp_select(all, K, lane);
+    for (int i = 0; i < P; ++i) all.k[i] = key[i];
+    all.k[P] = run;
+    return select_rounds<P + 1>(all, K, lane);
 }
 
 // Running top-K of x[0, n) taken by one warp in chunks of 32*P elements
 // (chunks seg0, seg0 + seg_stride, ...), merged into `run`.
+// With `synthetic` the row is not read: element j is taken to be (float)j,
+// which runs the common path of the selection on distinct values (used to
+// bring the code into the instruction cache ahead of the real call).
 template <int P, bool CG = false>
 __device__ __forceinline__ uint64_t warp_topk_fast(const float *x, int n, int K, int lane, int seg0,
-                                                   int seg_stride, uint64_t run, uint64_t *scratch) {
+                                                   int seg_stride, uint64_t run, uint64_t *scratch,
+                                                   bool synthetic = false) {
     for (int seg = seg0; (int64_t)seg * 32 * P < n; seg += seg_stride) {
         const int base = seg * 32 * P;
         float v[P];
 #pragma unroll
         for (int i = 0; i < P; ++i) {
             const int j = base + lane + 32 * i;
-            v[i] = j < n ? load_row<CG>(x, j) : 0.0f;
+            v[i] = j < n ? (synthetic ? (float)j : load_row<CG>(x, j)) : 0.0f;
         }
         uint64_t keys[P];
 #pragma unroll
