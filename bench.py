@@ -3,10 +3,10 @@
 One step = one pass of the router hot path over one batch: for each window
 size m in (1, 2, 4, 8, 16), A[m,2560] bf16 x W_r[2560,512] bf16 -> fp32 logits
 (weight streamed once) -> per-row top-10.  That is 31 rows per step.  The
-reported value is the two-launch form (one router_gemv_topk call per window
-with MR_ROUTER_TWO_LAUNCH: the GEMV kernel, then the top-k kernel); the fused
-form (one launch per window) is timed over the same K steps and printed
-beside it.  The weight comes from a
+reported value is the fused form, router_gemv_topk's default (one launch per
+window: the GEMV with the top-k as its tail); the two-launch form
+(MR_ROUTER_TWO_LAUNCH: the GEMV kernel, then the top-k kernel) is timed over
+the same K steps and printed beside it.  The weight comes from a
 rotating pool of copies larger than twice the L2, so every launch reads it
 from HBM.
 
@@ -53,6 +53,12 @@ def gemv_bytes(m: int, n: int, k: int) -> int:
     return n * k * 2 + m * k * 2 + m * n * 4
 
 
+def router_bytes(m: int) -> int:
+    """Algorithmic HBM bytes of one fused router window: W once, A once, and
+    the top-k indices and values (the logits are an intermediate)."""
+    return N_ROUTER * K_ROUTER * 2 + m * K_ROUTER * 2 + m * TOPK * 8
+
+
 def step_rows() -> int:
     return sum(WINDOWS)
 
@@ -70,6 +76,7 @@ def load_peaks():
 # Source files whose change invalidates a recorded ncu traffic figure.
 KERNEL_SOURCES = {
     "gemv_router": ("mrgemv.cu", "common.cuh", "topk_core.cuh"),
+    "router_fused": ("mrgemv.cu", "common.cuh", "topk_core.cuh"),
     "gemm": ("gemm_f16.cu", "common.cuh"),
 }
 
@@ -346,13 +353,12 @@ def run_gpu(args, world, rank, local):
     rb = RouterBench(device)
     flags = 0 if args.no_pdl else mr.MR_GEMV_PDL
     steps_per_cycle = max(1, rb.pool // len(WINDOWS))
-    # Two forms of the router step give identical outputs: two launches per
-    # window (the GEMV kernel, then the top-k kernel) and one fused launch.  `value` is always the two-launch form; the fused
-    # form is timed over the same K steps and printed beside it (on B200 its
-    # cross-CTA ticket and generation handshake costs more than the kernel
-    # boundary it removes).
-    forms = {"two_launch": rb.capture_steps(steps_per_cycle, flags, fused=False),
-             "fused": rb.capture_steps(steps_per_cycle, flags, fused=True)}
+    # Two forms of the router step give identical outputs: one fused launch
+    # per window (the API's default) and two launches (the GEMV kernel, then
+    # the top-k kernel).  `value` is always the fused form; the two-launch
+    # form is timed over the same K steps and printed beside it.
+    forms = {"fused": rb.capture_steps(steps_per_cycle, flags, fused=True),
+             "two_launch": rb.capture_steps(steps_per_cycle, flags, fused=False)}
     for g in forms.values():
         rb.time_graphs(g, max(args.warmup, 3))
     assert mr.mr_poll_errors() == 0
@@ -378,7 +384,7 @@ def run_gpu(args, world, rank, local):
         clocks[name] = clk.summary()
         clocks[name]["sampled_over_us"] = elapsed_us + sum(extra)
     errs = mr.mr_poll_errors()
-    best_form = "two_launch"
+    best_form = "fused"
     elapsed_max = form_us[best_form]
     # whole-job time per row: all ranks' rows over the slowest rank's time
     us_per_row = elapsed_max / (args.steps * step_rows() * world)
@@ -390,20 +396,32 @@ def run_gpu(args, world, rank, local):
     # ---- per-m curves and the GEMV roofline (back-to-back graph-captured calls)
     curves = gemv_curves(rb, flags, hbm_peak)
     curve = curves["router"]
-    # dominant kernel: the GEMV, averaged over the step's mix of m
+    # Dominant kernel: the fused router kernel (the step's only kernel),
+    # averaged over the step's mix of m.  Algorithmic bytes of a window: the
+    # weight once, A, and the top-10 indices and values; the logits stay an
+    # intermediate (in L2).  Its time: back-to-back graph-captured windows.
+    fused_us = sum(curve[str(m)]["router_fused_us_per_window"] for m in WINDOWS) / len(WINDOWS)
+    fused_bytes = sum(router_bytes(m) for m in WINDOWS) / len(WINDOWS)
+    achieved = fused_bytes / (fused_us * 1e3)
     mean_call_us = sum(curve[str(m)]["us_per_call"] for m in WINDOWS) / len(WINDOWS)
     mean_bytes = sum(gemv_bytes(m, N_ROUTER, K_ROUTER) for m in WINDOWS) / len(WINDOWS)
-    achieved = mean_bytes / (mean_call_us * 1e3)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": recorded_traffic("gemv_router"),
-                "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "mrgemv_bf16 (router, m mix 1..16)"}
+                "frac": achieved / hbm_peak, "traffic": recorded_traffic("router_fused"),
+                "peak_kind": f"{peak_kind} copy bandwidth",
+                "kernel": "router_gemv_topk fused kernel (GEMV + top-10 tail; router, m mix 1..16)",
+                "algorithmic_bytes_per_launch": fused_bytes, "us_per_launch": fused_us,
+                "gemv_only": {"kernel": "mrgemv_bf16 (router, m mix 1..16)",
+                              "achieved": mean_bytes / (mean_call_us * 1e3),
+                              "frac": mean_bytes / (mean_call_us * 1e3) / hbm_peak,
+                              "algorithmic_bytes_per_launch": mean_bytes, "us_per_launch": mean_call_us,
+                              "traffic": recorded_traffic("gemv_router")}}
     # The FFN and sweep weights (8.7 and 31 MB) are large enough to be HBM-bound:
     # their fractions of the measured copy bandwidth, m = 1..8, reported apart.
     roofline["by_shape_m1_to_8"] = {name: {m: curves[name][str(m)]["frac_of_measured_hbm"] for m in (1, 2, 4, 8)}
                                     for name, _, _ in GEMV_SHAPES}
 
     # ---- end to end through the public API with host buffers
-    e2e = run_e2e(rb, args, world, device, fused=False)
+    e2e = run_e2e(rb, args, world, device, fused=True)
 
     # ---- GEMM sweep (prompt-chunk shapes) and the m-sweep over both paths
     gemm = run_gemm_sweep(args) if not args.skip_gemm else None
@@ -993,6 +1011,18 @@ def profile_case(case: str):
         C = torch.empty((m, n), dtype=torch.float32, device="cuda")
         for i in range(3):
             mr.mrgemv_bf16(A[:m], W[i], C)
+    elif case == "fused":
+        # the fused router kernel alone, 4 launches per m, weight from DRAM
+        a16, w16 = synth.router(16)
+        pool = [torch.from_numpy(w16.view(np.int16)).cuda() for _ in range(110)]
+        A = torch.from_numpy(a16.view(np.int16)).cuda()
+        ws = torch.zeros(mr.router_gemv_topk_workspace_bytes(16, N_ROUTER, False) // 4 + 1,
+                         dtype=torch.int32, device="cuda")
+        for m in WINDOWS:
+            idx = torch.empty((m, TOPK), dtype=torch.int32, device="cuda")
+            val = torch.empty((m, TOPK), dtype=torch.float32, device="cuda")
+            for i in range(4):
+                mr.router_gemv_topk(A[:m], pool[(7 * i + m) % len(pool)], TOPK, idx, val, workspace=ws)
     elif case == "router_fused":
         a16, w16 = synth.router(16)
         pool = [torch.from_numpy(w16.view(np.int16)).cuda() for _ in range(110)]

@@ -43,7 +43,9 @@
 #include "topk_core.cuh"
 
 #include <algorithm>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 namespace mr {
 namespace gemv {
@@ -143,17 +145,26 @@ __device__ __forceinline__ void store_logit(const Params &p, int r, int col, flo
 // words: each segment's words are re-read until all carry the flag (bounded
 // by kWaitLimitNs; false if it runs out), then keyed and merged like
 // router_topk's rows.  `out`: lane t holds the rank-t key.
+// With `synthetic` the row is not read: word j is taken to be a ready
+// logit that grows with j, which runs the selection's common path (used to
+// bring the code into the instruction cache).
 template <int P>
 __device__ __forceinline__ bool tagged_topk(const uint64_t *row, int n, int K, int lane, uint64_t *scratch,
-                                            uint64_t &out) {
+                                            uint64_t &out, bool synthetic) {
     const uint64_t t0 = globaltimer_ns();
     uint64_t run = 0ull;
     for (int base = 0; base < n; base += 32 * P) {
         uint64_t w[P];
+        if (synthetic) {
 #pragma unroll
-        for (int i = 0; i < P; ++i) {
-            const int j = base + lane + 32 * i;
-            w[i] = j < n ? ld_relaxed_u64(row + j) : ((uint64_t)kTagReady << 32);
+            for (int i = 0; i < P; ++i)
+                w[i] = ((uint64_t)kTagReady << 32) | (0x3F800000u + (uint32_t)(base + lane + 32 * i));
+        } else {
+#pragma unroll
+            for (int i = 0; i < P; ++i) {
+                const int j = base + lane + 32 * i;
+                w[i] = j < n ? ld_relaxed_u64(row + j) : ((uint64_t)kTagReady << 32);
+            }
         }
         for (int spin = 0;; ++spin) {
             bool ready = true;
@@ -259,11 +270,14 @@ struct Smem {
     float *red;           // [groups][KW][MB x CG] k-slice partials (KW > 1)
 };
 
-// One column group: NC (power of two) columns of this warp's k-slice.
+// One column group: NC (power of two) columns of this warp's k-slice.  With
+// `warm` the group's code runs over whatever the slot holds, with no barrier
+// wait or arrival and no store: it only brings the instructions into the
+// instruction cache.
 template <int MB, int NC, int CGMAX, bool FUSED>
 __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g, int ncol,
                                          int col0, int slice, int lane, int q_begin, int q_end,
-                                         int chunk_groups) {
+                                         int chunk_groups, bool warm) {
     const int k = p.k;
     const int slot = g % p.S;
     // The first S groups come in up-front copy chunks (one barrier each,
@@ -271,7 +285,7 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     // the slot's refill barrier from phase 0.
     const uint64_t *bar = g < p.S ? &sm.chunk_full[g / chunk_groups] : &sm.full[slot];
     const uint32_t par = g < p.S ? 0u : (uint32_t)(g / p.S - 1) & 1u;
-    if (!mbar_wait_bounded(smem_u32(bar), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
+    if (!warm && !mbar_wait_bounded(smem_u32(bar), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
 
     const uint32_t w_s = launder(smem_u32(sm.ring + (size_t)slot * p.slot_bytes));
     const uint32_t a_s = launder(smem_u32(sm.a));
@@ -355,7 +369,7 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
         for (int j = 0; j < NC; ++j) asm volatile("" ::"f"(acc[rp][j].x), "f"(acc[rp][j].y));
     // This warp no longer reads the slot.
     __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&sm.empty[slot]));
+    if (lane == 0 && !warm) mbar_arrive(smem_u32(&sm.empty[slot]));
 
     constexpr int V = MB * NC;
     float v[V];
@@ -370,7 +384,9 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     ReduceScatter<V, 16>::run(v, lane, base);
     constexpr int PL = Scatter<V>::kPerLane;
 
-    if ((lane & Scatter<V>::kReplMask) == 0) {
+    // The warm pass stores nothing: the GEMV warps may already be using the
+    // partials' shared memory.
+    if ((lane & Scatter<V>::kReplMask) == 0 && !warm) {
         if (p.KW > 1) {
             // Partials of this k-slice for group g; the slices are summed, in
             // slice order, after every group of the CTA is done.
@@ -395,12 +411,13 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
 template <int MB, int NC, int CGMAX, bool FUSED>
 __device__ __forceinline__ bool run_group(const Params &p, const Smem &sm, int g, int ncol,
                                           int col0, int slice, int lane, int q_begin, int q_end,
-                                          int chunk_groups) {
+                                          int chunk_groups, bool warm) {
     if constexpr (NC > 1) {
         if (ncol <= NC / 2)
-            return run_group<MB, NC / 2, CGMAX, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups);
+            return run_group<MB, NC / 2, CGMAX, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end,
+                                                       chunk_groups, warm);
     }
-    return do_group<MB, NC, CGMAX, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups);
+    return do_group<MB, NC, CGMAX, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups, warm);
 }
 
 template <int MB, int CG, bool FUSED>
@@ -473,7 +490,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
             mbar_init(smem_u32(&sm.empty[s]), (uint32_t)p.KW);
         }
         mbar_init(smem_u32(sm.a_full), 1);
-        mbar_init(smem_u32(sm.parts_done), (uint32_t)(blockDim.x / 32));
+        mbar_init(smem_u32(sm.parts_done), (uint32_t)(p.KW * p.CWG));
         fence_mbar_init();
         // The whole first pass of the ring (min(ng, S) groups) is requested
         // now, before the wait for the previous kernel, in chunks of whole
@@ -484,81 +501,110 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     }
     // The weight stream is in flight; the next kernel may start launching.
     grid_launch_dependents();
-    // A may be produced by the previous kernel on the stream.
-    grid_dependency_wait();
-
-    // Stage A (bf16) in shared memory with one bulk copy (per row if strided);
-    // rows m..MB-1 are zero.  Under programmatic dependent launch the weight
-    // was requested while the previous kernel ran and has mostly landed by
-    // now.  (Per-thread cp.async copies of A measured slower: up to 3 us for
-    // 16 rows of 2560, since every CTA reads the same A lines.)
-    if (tid == 0) {
-        const uint32_t row_bytes = (uint32_t)k * 2u;
-        const uint32_t bar = smem_u32(sm.a_full);
-        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)p.m);
-        if (p.lda == k) {
-            bulk_g2s(smem_u32(sm.a), p.A, row_bytes * (uint32_t)p.m, bar);
-        } else {
-            for (int r = 0; r < p.m; ++r)
-                bulk_g2s(smem_u32(sm.a + (size_t)r * k), p.A + (int64_t)r * p.lda, row_bytes, bar);
-        }
-    }
-    {
-        const int chunks = k / 8;  // 16-byte chunks per row
-        for (int e = p.m * chunks + tid; e < MB * chunks; e += blockDim.x)
-            *reinterpret_cast<uint4 *>(sm.a + (size_t)(e / chunks) * k + 8 * (e % chunks)) =
-                make_uint4(0u, 0u, 0u, 0u);
-    }
-    __syncthreads();
-    bool failed = !mbar_wait_bounded(smem_u32(sm.a_full), 0u, MR_DEVERR_GEMV_TIMEOUT);
 
     const int slice = warp % p.KW;
     const int cw = warp / p.KW;
     const int q_total = k / 4;
     const int q_begin = (int)(((int64_t)slice * q_total) / p.KW);
     const int q_end = (int)(((int64_t)(slice + 1) * q_total) / p.KW);
+    constexpr int kQStep = 32 * q_unroll(MB, CG);  // one unrolled step of the k loop
 
-    for (int g = cw; g < ng && !failed; g += p.CWG) {
-        const int col0 = c_begin + g * CG;
-        const int ncol = min(CG, c_end - col0);
-        if (!run_group<MB, CG, CG, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups)) {
-            failed = true;
-            break;
+    // The GEMV warps are 0 .. KW * CWG - 1.  A launch with fewer than 16 of
+    // them has one more warp, which runs the code below once at kernel start
+    // ("warm"): the first group for one unrolled step of the k loop and the
+    // k-slice sum, over whatever shared memory holds, with no barrier wait
+    // or arrival and no global store, then exits.  It fetches the GEMV's
+    // instructions into the SM's instruction cache while the GEMV warps wait
+    // for the previous kernel and for A.  (A kernel's code starts cold when
+    // other kernels ran on the SM in between; measured at 1-2 us a call.)
+    // The GEMV warps run the same code (the same instructions) once, for real.
+    const int gemv_warps = p.KW * p.CWG;
+    const bool warm_warp = warp >= gemv_warps;
+    bool failed = false;
+#pragma unroll 1
+    for (int pass = warm_warp ? 0 : 1; pass < (warm_warp ? 1 : 2); ++pass) {
+        const bool warm = pass == 0;
+        if (!warm) {
+            // A may be produced by the previous kernel on the stream.
+            grid_dependency_wait();
+
+            // Stage A (bf16) in shared memory with one bulk copy (per row if
+            // strided); rows m..MB-1 are zero.  Under programmatic dependent
+            // launch the weight was requested while the previous kernel ran
+            // and has mostly landed by now.  (Per-thread cp.async copies of A
+            // measured slower: up to 3 us for 16 rows of 2560, since every
+            // CTA reads the same A lines.)
+            if (tid == 0) {
+                const uint32_t row_bytes = (uint32_t)k * 2u;
+                const uint32_t bar = smem_u32(sm.a_full);
+                mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)p.m);
+                if (p.lda == k) {
+                    bulk_g2s(smem_u32(sm.a), p.A, row_bytes * (uint32_t)p.m, bar);
+                } else {
+                    for (int r = 0; r < p.m; ++r)
+                        bulk_g2s(smem_u32(sm.a + (size_t)r * k), p.A + (int64_t)r * p.lda, row_bytes, bar);
+                }
+            }
+            {
+                const int chunks = k / 8;  // 16-byte chunks per row
+                for (int e = p.m * chunks + tid; e < MB * chunks; e += gemv_warps * 32)
+                    *reinterpret_cast<uint4 *>(sm.a + (size_t)(e / chunks) * k + 8 * (e % chunks)) =
+                        make_uint4(0u, 0u, 0u, 0u);
+            }
+            // The GEMV warps only (named barrier 1; the warm warp has left).
+            asm volatile("bar.sync 1, %0;" ::"r"(gemv_warps * 32) : "memory");
+            failed = !mbar_wait_bounded(smem_u32(sm.a_full), 0u, MR_DEVERR_GEMV_TIMEOUT);
         }
-        // Refill the slot with group g + S once every slice has released it.
-        // The whole warp waits (a lone lane in try_wait beside warp-mates
-        // suspended on another barrier can stall for the suspend time limit);
-        // lane 0 then issues the copies.
-        if (slice == 0 && g + p.S < ng) {
-            const int slot = g % p.S;
-            const uint32_t par = (uint32_t)(g / p.S) & 1u;
-            if (!mbar_wait_bounded(smem_u32(&sm.empty[slot]), par, MR_DEVERR_GEMV_TIMEOUT)) {
+
+        for (int g = warm ? 0 : cw; g < ng && !failed; g += p.CWG) {
+            const int col0 = c_begin + g * CG;
+            const int ncol = min(CG, c_end - col0);
+            if (!run_group<MB, CG, CG, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin,
+                                               warm ? min(q_end, q_begin + kQStep) : q_end, chunk_groups, warm)) {
                 failed = true;
                 break;
             }
-            if (lane == 0) issue_group(g + p.S);
-            __syncwarp();
+            if (warm) break;
+            // Refill the slot with group g + S once every slice has released
+            // it.  The whole warp waits (a lone lane in try_wait beside
+            // warp-mates suspended on another barrier can stall for the
+            // suspend time limit); lane 0 then issues the copies.
+            if (slice == 0 && g + p.S < ng) {
+                const int slot = g % p.S;
+                const uint32_t par = (uint32_t)(g / p.S) & 1u;
+                if (!mbar_wait_bounded(smem_u32(&sm.empty[slot]), par, MR_DEVERR_GEMV_TIMEOUT)) {
+                    failed = true;
+                    break;
+                }
+                if (lane == 0) issue_group(g + p.S);
+                __syncwarp();
+            }
         }
-    }
 
-    if (p.KW > 1) {
-        // Sum the k-slices of every output in slice order and store C; one
-        // barrier for the CTA instead of one handshake per group.
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(sm.parts_done));
-        if (!mbar_wait_bounded(smem_u32(sm.parts_done), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
-        constexpr int VCG = MB * CG;
-        for (int e = tid; e < ng * VCG; e += blockDim.x) {
-            const int g = e / VCG, rem = e % VCG;
-            const int r = rem / CG, col = c_begin + g * CG + rem % CG;
-            if (r < p.m && col < c_end) {
-                const float *src = sm.red + (size_t)g * p.KW * VCG + rem;
-                float acc = src[0];
-                for (int sl = 1; sl < p.KW; ++sl) acc = __fadd_rn(acc, src[(size_t)sl * VCG]);
-                store_logit<FUSED>(p, r, col, gate_out(p, acc));
+        if (p.KW > 1) {
+            // Sum the k-slices of every output in slice order and store C;
+            // one barrier for the CTA instead of one handshake per group.
+            __syncwarp();
+            if (!warm) {
+                if (lane == 0) mbar_arrive(smem_u32(sm.parts_done));
+                if (!mbar_wait_bounded(smem_u32(sm.parts_done), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
+            }
+            constexpr int VCG = MB * CG;
+            for (int e = warm ? lane : tid; e < ng * VCG; e += gemv_warps * 32) {
+                const int g = e / VCG, rem = e % VCG;
+                const int r = rem / CG, col = c_begin + g * CG + rem % CG;
+                if (r < p.m && col < c_end) {
+                    const float *src = sm.red + (size_t)g * p.KW * VCG + rem;
+                    float acc = src[0];
+                    for (int sl = 1; sl < p.KW; ++sl) acc = __fadd_rn(acc, src[(size_t)sl * VCG]);
+                    if (!warm) store_logit<FUSED>(p, r, col, gate_out(p, acc));
+                }
             }
         }
     }
+    // The warm warp goes on to warm the fused router's selection where this
+    // CTA selects a row.
+    if (warm_warp && !(FUSED && (int)blockIdx.x < p.m)) return;
 
     if constexpr (FUSED) {
         // Router top-k in the same launch, with no fence, counter or barrier
@@ -571,17 +617,19 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
         // storing only after this one has completed).  Only the <= m CTAs
         // that select wait, each after storing its own columns, so the other
         // CTAs always run to completion.
-        const int nwarps = blockDim.x >> 5;
+        // The warm warp runs the selection once on synthetic words.
+        const int nwarps = gemv_warps;
         // 64 keys of 16-byte aligned scratch per warp after the k-slice partials.
         const uintptr_t tk0 = reinterpret_cast<uintptr_t>(sm.red + red_floats(p.KW, ng_max_of(p.n, p.G, CG), MB, CG));
         uint64_t *tk = reinterpret_cast<uint64_t *>((tk0 + 15u) & ~(uintptr_t)15u) + warp * 64;
-        for (int r = (int)blockIdx.x + warp * p.G; r < p.m; r += nwarps * p.G) {
+        for (int r = warm_warp ? 0 : (int)blockIdx.x + warp * p.G; r < p.m; r += nwarps * p.G) {
             uint64_t *row = p.tags + (int64_t)r * p.n;
             uint64_t best = 0ull;
-            if (!tagged_topk<MR_FUSED_P>(row, p.n, p.topk, lane, tk, best)) {
+            if (!tagged_topk<MR_FUSED_P>(row, p.n, p.topk, lane, tk, best, warm_warp)) {
                 if (lane == 0) record_error(MR_DEVERR_GEMV_TIMEOUT);
                 return;
             }
+            if (warm_warp) return;
             if (lane < p.topk) {
                 const uint32_t j = topk::key_index(best);
                 p.idx[(int64_t)r * p.ldo + lane] = (int32_t)j;
@@ -644,6 +692,29 @@ cudaError_t ensure_attributes(int device) {
         }
     if (device >= 0 && device < 64) g_attr_done[device] = true;
     return cudaSuccess;
+}
+
+// Whether one more warp per CTA (the warm warp) keeps the CTAs per SM the
+// launch relies on: as many as without it, or at least two (this launch's CTA
+// beside the next launch's, or the two CTAs per SM of a split plan).  Asked of
+// the occupancy calculator once per (device, kernel, warps, shared memory).
+bool warm_warp_fits(KernelFn fn, int gemv_warps, size_t smem) {
+    if (gemv_warps >= kWarpsMax) return false;
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess) return false;
+    static std::mutex mu;
+    static std::map<std::tuple<int, const void *, int, size_t>, bool> cache;
+    const auto key = std::make_tuple(device, reinterpret_cast<const void *>(fn), gemv_warps, smem);
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    int without = 0, with = 0;
+    bool fits = false;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&without, fn, gemv_warps * 32, smem) == cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&with, fn, (gemv_warps + 1) * 32, smem) == cudaSuccess)
+        fits = with >= 1 && with >= std::min(without, 2);
+    cache[key] = fits;
+    return fits;
 }
 
 }  // namespace gemv
@@ -811,7 +882,10 @@ mr_status enqueue(const Params &p, const Plan &pl, uint32_t flags, bool fused, v
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.G);
-    cfg.blockDim = dim3((unsigned)(p.KW * p.CWG * 32));
+    // One warm warp beside the GEMV warps when the SM has room for it.
+    const KernelFn fn = kernel_for(pl.MB, pl.CG, fused);
+    const int warps = p.KW * p.CWG + (warm_warp_fits(fn, p.KW * p.CWG, pl.smem) ? 1 : 0);
+    cfg.blockDim = dim3((unsigned)(warps * 32));
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];
@@ -819,7 +893,7 @@ mr_status enqueue(const Params &p, const Plan &pl, uint32_t flags, bool fused, v
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = (flags & MR_GEMV_PDL) ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kernel_for(pl.MB, pl.CG, fused), p);
+    e = cudaLaunchKernelEx(&cfg, fn, p);
     return mr_host::cuda_status(e);
 }
 
