@@ -299,11 +299,11 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
 #pragma unroll
         for (int j = 0; j < NC; ++j) acc[rp][j] = make_float2(0.0f, 0.0f);
 
-    // The loads are software-pipelined by hand: the next row pair's A (or the
-    // next column's W, or the next chunk's first operands) is requested
-    // before the current FMAs issue, so one warp per scheduler does not wait
-    // out each shared-memory load.  The FMA sequence of every chain is the
-    // same as without pipelining.
+    // Operands come from shared memory through lds64 (non-volatile, so the
+    // compiler schedules the loads ahead of the FMAs that use them).  With
+    // fewer row pairs than columns the A operands of the chunk are loaded
+    // first and each column's W streams past them; otherwise the W operands
+    // are loaded first.  Either way every chain's FMA sequence is the same.
     auto a_at = [&](int r, int qq) { return lds64(a_s + (uint32_t)r * row_b + 8u * (uint32_t)qq); };
     auto w_at = [&](int j, int qq) { return lds64(w_s + (uint32_t)j * row_b + 8u * (uint32_t)qq); };
 #pragma unroll (q_unroll(MB, CGMAX))
