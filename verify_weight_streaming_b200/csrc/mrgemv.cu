@@ -107,6 +107,14 @@ struct Params {
 #ifndef MR_GEMV_KW_MAX
 #define MR_GEMV_KW_MAX 4
 #endif
+// Weight bytes a CTA requests before the dependency wait when its block is
+// larger than MR_GEMV_PREWAIT_SPLIT (smaller blocks are requested whole).
+#ifndef MR_GEMV_PREWAIT_BYTES
+#define MR_GEMV_PREWAIT_BYTES 65536u
+#endif
+#ifndef MR_GEMV_PREWAIT_SPLIT
+#define MR_GEMV_PREWAIT_SPLIT 98304u
+#endif
 __host__ __device__ inline int k_warps(int k) {
     const int q = k / 4;
     int best = 1;
@@ -448,6 +456,17 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
 
     // Groups per copy chunk when no slot is refilled (0 when slots are refilled).
     const int chunk_groups = (int)max(1u, (32768u + p.slot_bytes - 1) / p.slot_bytes);
+    // First-pass chunks requested before the dependency wait: all of them,
+    // except that a block larger than MR_GEMV_PREWAIT_SPLIT requests only
+    // MR_GEMV_PREWAIT_BYTES before the wait and the rest after A's copy, so
+    // that A does not queue behind the whole block (this CTA's copies are
+    // served in order, at ~44 GB/s per SM when every SM streams: 100 KB ahead
+    // of A delayed it by ~2 us).
+    const int first_chunks = (min(ng, p.S) + chunk_groups - 1) / chunk_groups;
+    const bool split_prewait = (size_t)ncols * (size_t)k * 2u > MR_GEMV_PREWAIT_SPLIT;
+    const int prewait_chunks =
+        split_prewait ? min(first_chunks, max(1, (int)(MR_GEMV_PREWAIT_BYTES / ((size_t)chunk_groups * p.slot_bytes))))
+                      : first_chunks;
     const int first = min(ng, p.S);
 
     auto issue_chunk = [&](int c) {
@@ -497,7 +516,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
         // groups of >= 32 KB each (small bulk copies stream below HBM
         // bandwidth: ~2.6 TB/s for 4 KB copies, ~6.2 TB/s for 16 KB, ~7 TB/s
         // for 32-64 KB).  The weight does not depend on the previous kernel.
-        for (int c = 0; c * chunk_groups < first; ++c) issue_chunk(c);
+        for (int c = 0; c < prewait_chunks; ++c) issue_chunk(c);
     }
     // The weight stream is in flight; the next kernel may start launching.
     grid_launch_dependents();
@@ -544,6 +563,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
                     for (int r = 0; r < p.m; ++r)
                         bulk_g2s(smem_u32(sm.a + (size_t)r * k), p.A + (int64_t)r * p.lda, row_bytes, bar);
                 }
+                for (int c = prewait_chunks; c < first_chunks; ++c) issue_chunk(c);
             }
             {
                 const int chunks = k / 8;  // 16-byte chunks per row
