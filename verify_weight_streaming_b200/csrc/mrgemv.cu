@@ -37,8 +37,9 @@
 //    share of the values), then the KW slices in slice order.  The tree of
 //    every output element is the same for every m, every row position and
 //    every column grouping, so row i is bitwise identical at every m.
-//  * Every wait is an mbarrier wait bounded in time; nothing uses bar.sync
-//    after the prologue, so a wait that runs out cannot strand other warps.
+//  * Every wait on data is an mbarrier wait bounded in time.  The GEMV warps
+//    meet at two named barriers (after A is staged, and before the k-slice
+//    sum), which every one of them reaches whether or not a wait ran out.
 #include "common.cuh"
 #include "topk_core.cuh"
 
@@ -274,7 +275,6 @@ struct Smem {
     uint64_t *full;       // [S] refills: slot s's uses 1, 2, ...
     uint64_t *empty;      // [S]
     uint64_t *a_full;     // [1] A has landed (A staged by a bulk copy)
-    uint64_t *parts_done; // [1] every warp has written its k-slice partials
     float *red;           // [groups][KW][MB x CG] k-slice partials (KW > 1)
 };
 
@@ -449,9 +449,8 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     sm.chunk_full = reinterpret_cast<uint64_t *>(sm.ring + (size_t)p.S * p.slot_bytes);
     sm.full = sm.chunk_full + p.S;
     sm.empty = sm.full + p.S;
-    uint64_t *misc = sm.empty + p.S;  // 6 words: two barriers and spare words
+    uint64_t *misc = sm.empty + p.S;  // 6 words: A's barrier and spare words
     sm.a_full = misc;
-    sm.parts_done = misc + 5;
     sm.red = reinterpret_cast<float *>(misc + 6);
 
     // Groups per copy chunk when no slot is refilled (0 when slots are refilled).
@@ -509,7 +508,6 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
             mbar_init(smem_u32(&sm.empty[s]), (uint32_t)p.KW);
         }
         mbar_init(smem_u32(sm.a_full), 1);
-        mbar_init(smem_u32(sm.parts_done), (uint32_t)(p.KW * p.CWG));
         fence_mbar_init();
         // The whole first pass of the ring (min(ng, S) groups) is requested
         // now, before the wait for the previous kernel, in chunks of whole
@@ -605,10 +603,9 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
             // Sum the k-slices of every output in slice order and store C;
             // one barrier for the CTA instead of one handshake per group.
             __syncwarp();
-            if (!warm) {
-                if (lane == 0) mbar_arrive(smem_u32(sm.parts_done));
-                if (!mbar_wait_bounded(smem_u32(sm.parts_done), 0u, MR_DEVERR_GEMV_TIMEOUT)) return;
-            }
+            // Named barrier 2 over the GEMV warps: each of them gets here
+            // (a failed wait only ends its group loop), so it cannot hang.
+            if (!warm) asm volatile("bar.sync 2, %0;" ::"r"(gemv_warps * 32) : "memory");
             constexpr int VCG = MB * CG;
             for (int e = warm ? lane : tid; e < ng * VCG; e += gemv_warps * 32) {
                 const int g = e / VCG, rem = e % VCG;
