@@ -155,3 +155,36 @@ def test_two_launch_flag_matches_fused_and_separate_calls(m, with_logits):
         assert np.array_equal(got.view(np.uint32), c_ref.view(np.uint32))
     with pytest.raises(mr.MrError):
         mr.router_gemv_topk(A, W, 10, idx, val, workspace=ws, flags=mr.MR_GEMV_SIGMOID)
+
+
+@pytest.mark.parametrize("heavy", [False, True])
+def test_fused_ties_inf_nan_through_the_tags(heavy):
+    """Special logits cross the tag array bit for bit: ties (equal W rows),
+    +-inf (an inf weight times a nonzero a) and NaN (inf times a zero a).
+    With `heavy`, 40 equal rows at the top leave more than 32 candidates, so
+    the selection takes its tie fallback inside the fused kernel."""
+    m, n, k = 4, 512, 64
+    a = synth.normal_bits(1400, (m, k), "bf16", 1.0)
+    w = synth.normal_bits(1401, (n, k), "bf16", 0.05)
+    top = range(100, 140) if heavy else (10, 300, 301)
+    w[5] = synth.normal_bits(1402, (1, k), "bf16", 1.0)[0]
+    for j in top:
+        w[j] = w[5]                      # equal logits: ties go to the lower index
+    w[7] = 0
+    w[7, 0] = 0x7F80                     # +inf weight
+    w[8] = 0
+    w[8, 1] = 0xFF80                     # -inf weight
+    a[2, 0] = 0                          # row 2: inf * 0 = NaN at column 7
+    A, W = dev_bits(a), dev_bits(w)
+    c_ref, i_ref, v_ref = two_launch(A, W, m, n, 10)
+    assert np.isnan(c_ref[2, 7]) and np.isinf(c_ref[0, 7]) and np.isinf(c_ref[0, 8])
+    ws = workspace(m, n, False)
+    idx = torch.full((m, 10), -1, dtype=torch.int32, device="cuda")
+    val = torch.full((m, 10), float("nan"), dtype=torch.float32, device="cuda")
+    mr.router_gemv_topk(A, W, 10, idx, val, workspace=ws, flags=mr.MR_GEMV_PDL)
+    assert np.array_equal(host(idx), i_ref)
+    assert np.array_equal(host(val).view(np.uint32), v_ref.view(np.uint32))
+    ri, rv = oracle.topk(c_ref, 10)
+    assert np.array_equal(host(idx), ri)
+    assert np.array_equal(host(val).view(np.uint32), rv.view(np.uint32))
+    assert tags_are_zero(ws, m, n)
