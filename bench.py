@@ -38,6 +38,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 WINDOWS = (1, 2, 4, 8, 16)
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e nominal bandwidth; fractions are also given against the measured copy
 K_ROUTER, N_ROUTER, TOPK = 2560, 512, 10
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -407,6 +408,7 @@ def run_gpu(args, world, rank, local):
     mean_bytes = sum(gemv_bytes(m, N_ROUTER, K_ROUTER) for m in WINDOWS) / len(WINDOWS)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": recorded_traffic("router_fused"),
+                "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                 "peak_kind": f"{peak_kind} copy bandwidth",
                 "kernel": "router_gemv_topk fused kernel (GEMV + top-10 tail; router, m mix 1..16)",
                 "algorithmic_bytes_per_launch": fused_bytes, "us_per_launch": fused_us,
@@ -419,6 +421,8 @@ def run_gpu(args, world, rank, local):
     # their fractions of the measured copy bandwidth, m = 1..8, reported apart.
     roofline["by_shape_m1_to_8"] = {name: {m: curves[name][str(m)]["frac_of_measured_hbm"] for m in (1, 2, 4, 8)}
                                     for name, _, _ in GEMV_SHAPES}
+    roofline["by_shape_m1_to_8_of_nominal_8tbs"] = {
+        name: {m: curves[name][str(m)]["GBps"] / NOMINAL_HBM_GBS for m in (1, 2, 4, 8)} for name, _, _ in GEMV_SHAPES}
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(rb, args, world, device, fused=True)
