@@ -1,6 +1,7 @@
 // Warp-level top-k under the total order of the router selection: value
 // descending, equal values by index ascending, -0.0 equal to +0.0, any NaN
-// above +inf.  Shared by router_topk and the fused router kernel.
+// above +inf.  Shared by router_topk, router_topk_merge and the fused router
+// kernel.
 #pragma once
 
 #include <stdint.h>
@@ -39,21 +40,12 @@ __device__ __forceinline__ float key_value(uint64_t key, bool &exact) {
     return __uint_as_float(b);
 }
 
-// Row loads: plain, or (CG) cached in L2 only, for rows other CTAs of the
-// same grid have just written (an L1 line cached earlier could be stale).
-template <bool CG>
-__device__ __forceinline__ float load_row(const float *x, int j) {
-    if constexpr (CG) return __ldcg(x + j);
-    return x[j];
-}
-
 // Value to report for a selected key: decoded from the key when that is
 // exact, else re-read from the row.
-template <bool CG = false>
 __device__ __forceinline__ float selected_value(uint64_t key, const float *x) {
     bool exact;
     const float v = key_value(key, exact);
-    return exact ? v : load_row<CG>(x, (int)key_index(key));
+    return exact ? v : x[key_index(key)];
 }
 
 // Sort L keys descending (insertion network, compile-time indices).
@@ -206,7 +198,7 @@ __device__ __forceinline__ uint64_t warp_topk_merge(uint64_t (&key)[P], uint64_t
 // With `synthetic` the row is not read: element j is taken to be (float)j,
 // which runs the common path of the selection on distinct values (used to
 // bring the code into the instruction cache ahead of the real call).
-template <int P, bool CG = false>
+template <int P>
 __device__ __forceinline__ uint64_t warp_topk_fast(const float *x, int n, int K, int lane, int seg0,
                                                    int seg_stride, uint64_t run, uint64_t *scratch,
                                                    bool synthetic = false) {
@@ -216,7 +208,7 @@ __device__ __forceinline__ uint64_t warp_topk_fast(const float *x, int n, int K,
 #pragma unroll
         for (int i = 0; i < P; ++i) {
             const int j = base + lane + 32 * i;
-            v[i] = j < n ? (synthetic ? (float)j : load_row<CG>(x, j)) : 0.0f;
+            v[i] = j < n ? (synthetic ? (float)j : x[j]) : 0.0f;
         }
         uint64_t keys[P];
 #pragma unroll
