@@ -7,19 +7,25 @@
 // fall with m because the weight bytes are not re-streamed per row.
 //
 // Design (B200):
-//  * grid = one CTA per SM (at most n); CTA b owns the contiguous column block
-//    [b*n/G, (b+1)*n/G) of Wt, i.e. a contiguous run of weight rows.
+//  * grid = one CTA per SM (at most n; two per SM for large blocks under
+//    PDL); CTA b owns the contiguous column block [b*n/G, (b+1)*n/G) of Wt,
+//    i.e. a contiguous run of weight rows.
 //  * The block streams through a ring of shared-memory slots, one column group
 //    (up to CG columns x k) per slot, with cp.async.bulk global->shared copies
 //    counted on an mbarrier (no tensor map; each copy lands in its own CTA).
 //    Group g is consumed by column warp g % CWG from slot g % S; when slots
 //    are refilled, S is a multiple of CWG, so each slot has a single consumer
-//    warp that waits for the slot's successive uses in order.  The whole first
-//    pass of the ring is requested before griddepcontrol.wait, so under
+//    warp that waits for the slot's successive uses in order.  The first
+//    pass of the ring is requested before griddepcontrol.wait (up to 64 KB
+//    of it for blocks over 96 KB, the rest right after A), so under
 //    programmatic dependent launch the weight streams while the previous
 //    kernel runs.
 //  * KW x CWG warps per CTA, at most 16.  More warps than k-slices work on
-//    separate column groups in parallel.
+//    separate column groups in parallel.  One more warp, where the SM has
+//    room, runs the same code once at kernel start without storing anything,
+//    to bring it into the instruction cache (the warm warp).
+//  * Fused router (router_gemv_topk): every logit is also stored as a flagged
+//    64-bit word; CTA r polls row r's words and selects its top-k.
 //  * A (m rows, bf16) is staged once in shared memory by a bulk copy issued
 //    after the grid-dependency wait; rows m..MB-1 are zero.
 //  * The k loop reads shared memory with loads the compiler may schedule
