@@ -109,9 +109,13 @@ mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw
  * mrgemv_bf16_plan -- the launch plan mrgemv_bf16_ex would use for (m, n, k,
  * flags) on a device with sm_count SMs and smem_optin bytes of opt-in shared
  * memory per block (pure host arithmetic, no CUDA call).  out[8] receives:
- * grid CTAs, threads per CTA, dynamic shared bytes, weight ring slots, warps
- * splitting k, column-group warps, row bucket (m rounded up to 1/2/4/8/16),
- * columns per group.  Size errors are reported as by mrgemv_bf16.
+ * grid CTAs, threads of the GEMV warps per CTA, dynamic shared bytes, weight
+ * ring slots, warps splitting k, column-group warps, row bucket (m rounded up
+ * to 1/2/4/8/16), columns per group.  At launch, where the occupancy
+ * calculator allows, a CTA gets one more warp that only fetches the code
+ * ahead (it computes and stores nothing), and the fused router's 16-row
+ * bucket splits each column group's rows over two warps; neither changes an
+ * output bit.  Size errors are reported as by mrgemv_bf16.
  */
 mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t flags, int32_t sm_count,
                            int32_t smem_optin, int32_t *out);
