@@ -113,9 +113,8 @@ mr_status mrgemv_bf16_ex(const void *A, int64_t lda, const void *Wt, int64_t ldw
  * ring slots, warps splitting k, column-group warps, row bucket (m rounded up
  * to 1/2/4/8/16), columns per group.  At launch, where the occupancy
  * calculator allows, a CTA gets one more warp that only fetches the code
- * ahead (it computes and stores nothing), and the fused router's 16-row
- * bucket splits each column group's rows over two warps; neither changes an
- * output bit.  Size errors are reported as by mrgemv_bf16.
+ * ahead (it stores nothing and changes no output bit).  Size errors are
+ * reported as by mrgemv_bf16.
  */
 mr_status mrgemv_bf16_plan(int32_t m, int32_t n, int32_t k, uint32_t flags, int32_t sm_count,
                            int32_t smem_optin, int32_t *out);

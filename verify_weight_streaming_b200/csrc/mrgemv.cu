@@ -92,8 +92,6 @@ struct Params {
     int KW;         // warps splitting k (function of k only)
     int CWG;        // column-group warps per CTA
     int S;          // ring slots
-    int RW;         // warps splitting the rows of a column group (1 or 2)
-    int MBT;        // row bucket of the launch (RW x the kernel's rows per warp)
     uint32_t a_bytes;     // shared bytes reserved for A (MB rows)
     uint32_t slot_bytes;  // CG * k * 2
     int sigmoid;          // store 1 / (1 + exp(-c)) instead of c (MR_GEMV_SIGMOID)
@@ -118,9 +116,6 @@ struct Params {
 #endif
 // Weight bytes a CTA requests before the dependency wait when its block is
 // larger than MR_GEMV_PREWAIT_SPLIT (smaller blocks are requested whole).
-#ifndef MR_GEMV_ROW_SPLIT
-#define MR_GEMV_ROW_SPLIT 1  // fused router, 16-row bucket: split a group's rows over two warps when the SM has room
-#endif
 #ifndef MR_GEMV_PREWAIT_BYTES
 #define MR_GEMV_PREWAIT_BYTES 65536u
 #endif
@@ -295,7 +290,7 @@ struct Smem {
 // instruction cache.
 template <int MB, int NC, int CGMAX, bool FUSED>
 __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g, int ncol,
-                                         int col0, int slice, int r0, int lane, int q_begin, int q_end,
+                                         int col0, int slice, int lane, int q_begin, int q_end,
                                          int chunk_groups, bool warm) {
     const int k = p.k;
     const int slot = g % p.S;
@@ -307,7 +302,7 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     if (!warm && !mbar_wait_bounded(smem_u32(bar), par, MR_DEVERR_GEMV_TIMEOUT)) return false;
 
     const uint32_t w_s = launder(smem_u32(sm.ring + (size_t)slot * p.slot_bytes));
-    const uint32_t a_s = launder(smem_u32(sm.a + (size_t)r0 * k));  // this warp's MB rows
+    const uint32_t a_s = launder(smem_u32(sm.a));
     const uint32_t row_b = (uint32_t)k * 2u;
     // acc[rp][j] holds rows (2rp, 2rp+1) of column j: one fp32 chain per
     // (row, column), over this lane's k positions in ascending order.
@@ -409,17 +404,17 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
         if (p.KW > 1) {
             // Partials of this k-slice for group g; the slices are summed, in
             // slice order, after every group of the CTA is done.
-            float *red = sm.red + ((size_t)g * p.KW + slice) * ((size_t)p.MBT * CGMAX);
+            float *red = sm.red + ((size_t)g * p.KW + slice) * (MB * CGMAX);
 #pragma unroll
             for (int i = 0; i < PL; ++i) {
                 const int idx = base + i;
-                red[(r0 + idx / NC) * CGMAX + idx % NC] = v[i];
+                red[(idx / NC) * CGMAX + idx % NC] = v[i];
             }
         } else {
 #pragma unroll
             for (int i = 0; i < PL; ++i) {
                 const int idx = base + i;
-                const int r = r0 + idx / NC, j = idx % NC;
+                const int r = idx / NC, j = idx % NC;
                 if (r < p.m && j < ncol) store_logit<FUSED>(p, r, col0 + j, gate_out(p, v[i]));
             }
         }
@@ -429,15 +424,14 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
 
 template <int MB, int NC, int CGMAX, bool FUSED>
 __device__ __forceinline__ bool run_group(const Params &p, const Smem &sm, int g, int ncol,
-                                          int col0, int slice, int r0, int lane, int q_begin, int q_end,
+                                          int col0, int slice, int lane, int q_begin, int q_end,
                                           int chunk_groups, bool warm) {
     if constexpr (NC > 1) {
         if (ncol <= NC / 2)
-            return run_group<MB, NC / 2, CGMAX, FUSED>(p, sm, g, ncol, col0, slice, r0, lane, q_begin, q_end,
+            return run_group<MB, NC / 2, CGMAX, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end,
                                                        chunk_groups, warm);
     }
-    return do_group<MB, NC, CGMAX, FUSED>(p, sm, g, ncol, col0, slice, r0, lane, q_begin, q_end, chunk_groups,
-                                          warm);
+    return do_group<MB, NC, CGMAX, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin, q_end, chunk_groups, warm);
 }
 
 template <int MB, int CG, bool FUSED>
@@ -517,7 +511,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
         for (int s = 0; s < p.S; ++s) {
             mbar_init(smem_u32(&sm.chunk_full[s]), 1);
             mbar_init(smem_u32(&sm.full[s]), 1);
-            mbar_init(smem_u32(&sm.empty[s]), (uint32_t)(p.KW * p.RW));
+            mbar_init(smem_u32(&sm.empty[s]), (uint32_t)p.KW);
         }
         mbar_init(smem_u32(sm.a_full), 1);
         fence_mbar_init();
@@ -531,11 +525,8 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     // The weight stream is in flight; the next kernel may start launching.
     grid_launch_dependents();
 
-    // warp = slice + KW * (row half + RW * column warp): KW k-slices, RW row
-    // halves (MB rows each) and CWG column warps.
     const int slice = warp % p.KW;
-    const int r0 = ((warp / p.KW) % p.RW) * MB;
-    const int cw = warp / (p.KW * p.RW);
+    const int cw = warp / p.KW;
     const int q_total = k / 4;
     const int q_begin = (int)(((int64_t)slice * q_total) / p.KW);
     const int q_end = (int)(((int64_t)(slice + 1) * q_total) / p.KW);
@@ -550,7 +541,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     // for the previous kernel and for A.  (A kernel's code starts cold when
     // other kernels ran on the SM in between; measured at 1-2 us a call.)
     // The GEMV warps run the same code (the same instructions) once, for real.
-    const int gemv_warps = p.KW * p.CWG * p.RW;
+    const int gemv_warps = p.KW * p.CWG;
     const bool warm_warp = warp >= gemv_warps;
     bool failed = false;
 #pragma unroll 1
@@ -580,7 +571,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
             }
             {
                 const int chunks = k / 8;  // 16-byte chunks per row
-                for (int e = p.m * chunks + tid; e < p.MBT * chunks; e += gemv_warps * 32)
+                for (int e = p.m * chunks + tid; e < MB * chunks; e += gemv_warps * 32)
                     *reinterpret_cast<uint4 *>(sm.a + (size_t)(e / chunks) * k + 8 * (e % chunks)) =
                         make_uint4(0u, 0u, 0u, 0u);
             }
@@ -592,7 +583,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
         for (int g = warm ? 0 : cw; g < ng && !failed; g += p.CWG) {
             const int col0 = c_begin + g * CG;
             const int ncol = min(CG, c_end - col0);
-            if (!run_group<MB, CG, CG, FUSED>(p, sm, g, ncol, col0, slice, r0, lane, q_begin,
+            if (!run_group<MB, CG, CG, FUSED>(p, sm, g, ncol, col0, slice, lane, q_begin,
                                                warm ? min(q_end, q_begin + kQStep) : q_end, chunk_groups, warm)) {
                 failed = true;
                 break;
@@ -602,7 +593,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
             // it.  The whole warp waits (a lone lane in try_wait beside
             // warp-mates suspended on another barrier can stall for the
             // suspend time limit); lane 0 then issues the copies.
-            if (slice == 0 && r0 == 0 && g + p.S < ng) {
+            if (slice == 0 && g + p.S < ng) {
                 const int slot = g % p.S;
                 const uint32_t par = (uint32_t)(g / p.S) & 1u;
                 if (!mbar_wait_bounded(smem_u32(&sm.empty[slot]), par, MR_DEVERR_GEMV_TIMEOUT)) {
@@ -621,7 +612,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
             // Named barrier 2 over the GEMV warps: each of them gets here
             // (a failed wait only ends its group loop), so it cannot hang.
             if (!warm) asm volatile("bar.sync 2, %0;" ::"r"(gemv_warps * 32) : "memory");
-            const int VCG = p.MBT * CG;
+            constexpr int VCG = MB * CG;
             for (int e = warm ? lane : tid; e < ng * VCG; e += gemv_warps * 32) {
                 const int g = e / VCG, rem = e % VCG;
                 const int r = rem / CG, col = c_begin + g * CG + rem % CG;
@@ -652,8 +643,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
         // The warm warp runs the selection once on synthetic words.
         const int nwarps = gemv_warps;
         // 64 keys of 16-byte aligned scratch per warp after the k-slice partials.
-        const uintptr_t tk0 =
-            reinterpret_cast<uintptr_t>(sm.red + red_floats(p.KW, ng_max_of(p.n, p.G, CG), p.MBT, CG));
+        const uintptr_t tk0 = reinterpret_cast<uintptr_t>(sm.red + red_floats(p.KW, ng_max_of(p.n, p.G, CG), MB, CG));
         uint64_t *tk = reinterpret_cast<uint64_t *>((tk0 + 15u) & ~(uintptr_t)15u) + warp * 64;
         for (int r = warm_warp ? 0 : (int)blockIdx.x + warp * p.G; r < p.m; r += nwarps * p.G) {
             uint64_t *row = p.tags + (int64_t)r * p.n;
@@ -725,28 +715,6 @@ cudaError_t ensure_attributes(int device) {
         }
     if (device >= 0 && device < 64) g_attr_done[device] = true;
     return cudaSuccess;
-}
-
-// Whether splitting each column group's rows over two warps (the half-bucket
-// kernel `half` with twice the warps) keeps the CTAs per SM of the unsplit
-// launch, or at least two.  Asked once per (device, kernels, warps, shared
-// memory).
-bool row_split_fits(KernelFn full, KernelFn half, int gemv_warps, size_t smem) {
-    int device = 0;
-    if (cudaGetDevice(&device) != cudaSuccess) return false;
-    static std::mutex mu;
-    static std::map<std::tuple<int, const void *, int, size_t>, bool> cache;
-    const auto key = std::make_tuple(device, reinterpret_cast<const void *>(full), gemv_warps, smem);
-    std::lock_guard<std::mutex> lock(mu);
-    const auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
-    int unsplit = 0, split = 0;
-    bool fits = false;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&unsplit, full, gemv_warps * 32, smem) == cudaSuccess &&
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&split, half, 2 * gemv_warps * 32, smem) == cudaSuccess)
-        fits = split >= 1 && split >= std::min(unsplit, 2);
-    cache[key] = fits;
-    return fits;
 }
 
 // Whether one more warp per CTA (the warm warp) keeps the CTAs per SM the
@@ -914,8 +882,6 @@ mr_status prepare(const void *A, int64_t lda, const void *Wt, int64_t ldw, float
     p.KW = pl.KW;
     p.CWG = pl.CWG;
     p.S = pl.S;
-    p.RW = 1;  // the row split is chosen at launch (it depends on the device)
-    p.MBT = pl.MB;
     p.a_bytes = pl.a_bytes;
     p.slot_bytes = pl.slot_bytes;
     p.sigmoid = (flags & MR_GEMV_SIGMOID) ? 1 : 0;
@@ -930,7 +896,7 @@ mr_status prepare(const void *A, int64_t lda, const void *Wt, int64_t ldw, float
 }
 
 // Launch a prepared plan on `stream`.
-mr_status enqueue(Params p, const Plan &pl, uint32_t flags, bool fused, void *stream) {
+mr_status enqueue(const Params &p, const Plan &pl, uint32_t flags, bool fused, void *stream) {
     int device = 0;
     cudaError_t e = cudaGetDevice(&device);
     if (e != cudaSuccess) return mr_host::cuda_status(e);
@@ -939,25 +905,9 @@ mr_status enqueue(Params p, const Plan &pl, uint32_t flags, bool fused, void *st
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.G);
-    // The fused router's 16-row bucket splits its rows over two warps per
-    // (k-slice, column group) where that fits: m = 16 windows 6.55 -> 5.92 us.
-    // Not the plain GEMV: a top-k kernel launched early after it (the
-    // two-launch router, or router_topk after mrgemv_bf16) then finds no
-    // registers beside two GEMV CTAs per SM (that window went 6.45 -> 7.79 us).
-    const int gw1 = p.KW * p.CWG;
-    p.RW = 1;
-    p.MBT = pl.MB;
-    KernelFn fn = kernel_for(pl.MB, pl.CG, fused);
-    if (MR_GEMV_ROW_SPLIT && fused && pl.MB >= 16 && 2 * gw1 <= kWarpsMax) {
-        const KernelFn half = kernel_for(pl.MB / 2, pl.CG, fused);
-        if (row_split_fits(fn, half, gw1, pl.smem)) {
-            p.RW = 2;
-            fn = half;
-        }
-    }
     // One warm warp beside the GEMV warps when the SM has room for it.
-    const int gw = gw1 * p.RW;
-    const int warps = gw + (warm_warp_fits(fn, gw, pl.smem) ? 1 : 0);
+    const KernelFn fn = kernel_for(pl.MB, pl.CG, fused);
+    const int warps = p.KW * p.CWG + (warm_warp_fits(fn, p.KW * p.CWG, pl.smem) ? 1 : 0);
     cfg.blockDim = dim3((unsigned)(warps * 32));
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
