@@ -122,6 +122,66 @@ def test_rows_bitwise_identical_across_m(shape):
         assert np.array_equal(single.view(np.uint32), full[i:i + 1].view(np.uint32))
 
 
+# Row buckets of 1-2 rows advance two rows per packed fp32 FMA on converted
+# operands; buckets of 4 and more use the mixed-precision FMA on the bf16
+# operands.  The two are the same arithmetic, which these check on the values
+# where hardware shortcuts would show: subnormals, infinities and NaN.
+_SMALL_POW2 = np.array([0x0000, 0x3F80, 0xBF80, 0x4000, 0xC000, 0x4080, 0xC080], np.uint16)  # 0, +-1, +-2, +-4
+
+
+def _subnormal_bits(rng, shape):
+    """bf16 subnormals: exponent field 0, mantissa 1..127, either sign."""
+    return ((rng.integers(0, 2, size=shape) << 15) | rng.integers(1, 128, size=shape)).astype(np.uint16)
+
+
+@pytest.mark.parametrize("side", ["A", "W"])
+def test_subnormal_operands_are_exact_at_every_m(side):
+    """Subnormal bf16 times 0, +-1, +-2 or +-4: every product and partial sum is
+    a multiple of 2^-133 with fewer than 2^24 of them, so the fp32 result is
+    exact (no operand or result may be flushed to zero), at every m."""
+    rng = np.random.default_rng(41 if side == "A" else 42)
+    m_max, n, k = 16, 40, 264
+    if side == "A":
+        a = _subnormal_bits(rng, (m_max, k))
+        w = _SMALL_POW2[rng.integers(0, len(_SMALL_POW2), size=(n, k))]
+    else:
+        a = _SMALL_POW2[rng.integers(0, len(_SMALL_POW2), size=(m_max, k))]
+        w = _subnormal_bits(rng, (n, k))
+    for m in (1, 2, 3, 4, 5, 8, 9, 16):
+        c = run_gemv(a[:m], w)
+        c64, _ = oracle.matmul(a[:m], "bf16", w, "bf16")
+        assert np.count_nonzero(c64) > m * n // 2
+        assert np.array_equal(c.astype(np.float64), c64), f"m={m}"
+
+
+def test_inf_nan_rows_bitwise_identical_across_m():
+    """Infinities and NaN in A and W: the same bits at every m (NaN included),
+    and NaN / +-inf exactly where the oracle has them."""
+    k, n = 520, 96
+    a = synth.normal_bits(51, (16, k), "bf16", 1.0)
+    w = synth.normal_bits(52, (n, k), "bf16", 1.0 / np.sqrt(k))
+    a[1, 7] = 0x7F80    # +inf: row 1 is +-inf or NaN wherever W[:, 7] != 0
+    a[4, 100] = 0xFF80  # -inf
+    a[4, 300] = 0x7F80  # and +inf in the same row: NaN where both products are finite-signed
+    a[6, 9] = 0x7FC0    # NaN
+    a[11, 513] = 0xFFC1  # NaN with a payload and the sign set
+    w[3, 200] = 0x7F80  # column 3: +inf in every row with a nonzero A[:, 200]
+    w[50, 17] = 0x0000
+    a[13, 17] = 0x7F80  # inf times zero in column 50: NaN
+    full = run_gemv(a, w)
+    c64, _ = oracle.matmul(a, "bf16", w, "bf16")
+    assert np.array_equal(np.isnan(full), np.isnan(c64))
+    assert np.array_equal(np.isposinf(full), np.isposinf(c64))
+    assert np.array_equal(np.isneginf(full), np.isneginf(c64))
+    assert np.isnan(full).any() and np.isinf(full).any()
+    for m in range(1, 16):
+        part = run_gemv(a[:m], w)
+        assert np.array_equal(part.view(np.uint32), full[:m].view(np.uint32)), f"m={m}"
+    for i in (1, 4, 6, 11, 13):
+        single = run_gemv(a[i:i + 1], w)
+        assert np.array_equal(single.view(np.uint32), full[i:i + 1].view(np.uint32)), f"row {i}"
+
+
 def test_pdl_flag_gives_identical_bits():
     a, w = synth.router(8)
     plain = run_gemv(a, w)

@@ -31,13 +31,14 @@
 //  * The k loop reads shared memory with loads the compiler may schedule
 //    freely (their addresses pass through a volatile move after the slot's
 //    barrier wait, and every accumulator is pinned before the slot is
-//    released), and advances two rows' chains per fma.rn.f32x2.
+//    released), and advances every chain with fma.rn.f32.bf16 on the bf16
+//    operands as they are in shared memory (one rounding in fp32: the same
+//    bits as an fp32 FMA of the converted values, with no conversions).
 //  * Lanes split k in 4-element chunks: chunk q belongs to lane q % 32 of the
 //    k-slice that holds it.  KW warps split k into contiguous slices; KW is a
 //    function of k alone.  Each lane keeps one fp32 accumulator per (row,
-//    column), updated in ascending k; rows are paired so that one
-//    fma.rn.f32x2 advances two rows' chains (a single row runs with a zero
-//    partner row).
+//    column), updated in ascending k.  Rows run in buckets of 1, 2, 4, 8 or
+//    16 (a bucket's spare rows are zero).
 //  * Reduction: a fixed xor-butterfly over the 32 lanes
 //    (bit 16, 8, 4, 2, 1; realised as a reduce-scatter so each lane finishes a
 //    share of the values), then the KW slices in slice order.  The tree of
@@ -59,17 +60,15 @@ namespace gemv {
 
 // Warps per CTA at most (512 threads, so at most 128 registers each: a CTA
 // of fewer warps then leaves room on its SM for the next launch's CTA), and
-// the unroll of the k loop.  None of this changes an output's arithmetic: a
-// lane's chain and the reduction order are fixed by k.
-#ifndef MR_GEMV_UNROLL_SMALL
-#define MR_GEMV_UNROLL_SMALL 2
-#endif
-#ifndef MR_GEMV_UNROLL_LARGE
-#define MR_GEMV_UNROLL_LARGE 1
-#endif
+// the unroll of the k loop: two steps, except for 8-column groups of 4 or more
+// rows and for 16 rows, whose accumulators leave few registers for a second
+// step (measured: one step is faster there, two elsewhere).  None of this
+// changes an output's arithmetic: a lane's chain and the reduction order are
+// fixed by k.
 constexpr int kWarpsMax = 16;
 __host__ __device__ constexpr int warps_max(int, int) { return kWarpsMax; }
-__host__ __device__ constexpr int q_unroll(int MB, int) { return MB >= 8 ? MR_GEMV_UNROLL_LARGE : MR_GEMV_UNROLL_SMALL; }
+__host__ __device__ constexpr int q_unroll(int MB, int CG) { return ((CG >= 8 && MB >= 4) || MB >= 16) ? 1 : 2; }
+
 constexpr int kMaxRows = 16;
 // Fused router: each logit is also stored as one 64-bit word, the flag
 // kTagReady in the high half and the logit's bits in the low half, in a tag
@@ -203,8 +202,6 @@ __device__ __forceinline__ bool tagged_topk(const uint64_t *row, int n, int K, i
     return true;
 }
 
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // 8-byte load from shared memory by 32-bit shared address (always LDS, never
 // a generic load).  Not volatile: the compiler may schedule it like any
@@ -225,9 +222,22 @@ __device__ __forceinline__ uint32_t launder(uint32_t x) {
     return y;
 }
 
-// acc.x = fma(a.x, b.x, acc.x); acc.y = fma(a.y, b.y, acc.y): two independent
-// round-to-nearest fp32 FMAs in one instruction (fma.rn.f32x2).
-__device__ __forceinline__ void ffma2(float2 &acc, float2 a, float2 b) { acc = __ffma2_rn(a, b, acc); }
+// acc = fma(a_h, w_h, acc) with a_h, w_h the bf16 in half H (0 low, 1 high) of
+// a and w, multiplied and added in one rounding to nearest in fp32.  A bf16
+// converts to fp32 exactly and the product of two bf16 is exact in fp32, so
+// this is bit for bit the fp32 FMA of the converted operands, without the
+// conversions.
+template <int H>
+__device__ __forceinline__ void fma_bf16(float &acc, uint32_t a, uint32_t w) {
+    if constexpr (H == 0)
+        asm("{\n\t.reg .b16 al, ah, wl, wh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {wl, wh}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, al, wl, %0;\n\t}"
+            : "+f"(acc) : "r"(a), "r"(w));
+    else
+        asm("{\n\t.reg .b16 al, ah, wl, wh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {wl, wh}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, ah, wh, %0;\n\t}"
+            : "+f"(acc) : "r"(a), "r"(w));
+}
 
 // Reduce-scatter over the warp: level D pairs lanes that differ in bit D (16,
 // 8, 4, 2, 1 in that order).  While more than one value is left, the lane with
@@ -304,83 +314,52 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     const uint32_t w_s = launder(smem_u32(sm.ring + (size_t)slot * p.slot_bytes));
     const uint32_t a_s = launder(smem_u32(sm.a));
     const uint32_t row_b = (uint32_t)k * 2u;
-    // acc[rp][j] holds rows (2rp, 2rp+1) of column j: one fp32 chain per
-    // (row, column), over this lane's k positions in ascending order.
-    constexpr int RP = MB / 2;
-    float2 acc[RP][NC];
+    // acc[r][j]: one fp32 chain per (row, column), over this lane's k
+    // positions in ascending order.
+    float acc[MB][NC];
 #pragma unroll
-    for (int rp = 0; rp < RP; ++rp)
+    for (int r = 0; r < MB; ++r)
 #pragma unroll
-        for (int j = 0; j < NC; ++j) acc[rp][j] = make_float2(0.0f, 0.0f);
+        for (int j = 0; j < NC; ++j) acc[r][j] = 0.0f;
 
     // Operands come from shared memory through lds64 (non-volatile, so the
-    // compiler schedules the loads ahead of the FMAs that use them).  With
-    // fewer row pairs than columns the A operands of the chunk are loaded
-    // first and each column's W streams past them; otherwise the W operands
-    // are loaded first.  Either way every chain's FMA sequence is the same.
+    // compiler schedules the loads ahead of the FMAs that use them): four k
+    // positions of every row of A and every column of the group.  At each of
+    // the four positions, in order, every (row, column) chain advances by one
+    // mixed-precision FMA, so consecutive FMAs are independent of each other.
     auto a_at = [&](int r, int qq) { return lds64(a_s + (uint32_t)r * row_b + 8u * (uint32_t)qq); };
     auto w_at = [&](int j, int qq) { return lds64(w_s + (uint32_t)j * row_b + 8u * (uint32_t)qq); };
 #pragma unroll (q_unroll(MB, CGMAX))
     for (int q = q_begin + lane; q < q_end; q += 32) {
-        if constexpr (RP < NC) {
-            float2 ap[RP][4];
+        uint2 wr[NC], ar[MB];
 #pragma unroll
-            for (int rp = 0; rp < RP; ++rp) {
-                const uint2 r0 = a_at(2 * rp, q), r1 = a_at(2 * rp + 1, q);
-                ap[rp][0] = make_float2(bf16lo(r0.x), bf16lo(r1.x));
-                ap[rp][1] = make_float2(bf16hi(r0.x), bf16hi(r1.x));
-                ap[rp][2] = make_float2(bf16lo(r0.y), bf16lo(r1.y));
-                ap[rp][3] = make_float2(bf16hi(r0.y), bf16hi(r1.y));
-            }
+        for (int j = 0; j < NC; ++j) wr[j] = w_at(j, q);
 #pragma unroll
-            for (int j = 0; j < NC; ++j) {
-                const uint2 raw = w_at(j, q);
-                const float w0 = bf16lo(raw.x), w1 = bf16hi(raw.x), w2 = bf16lo(raw.y), w3 = bf16hi(raw.y);
-                const float2 d0 = make_float2(w0, w0), d1 = make_float2(w1, w1), d2 = make_float2(w2, w2),
-                             d3 = make_float2(w3, w3);
+        for (int r = 0; r < MB; ++r) ar[r] = a_at(r, q);
 #pragma unroll
-                for (int rp = 0; rp < RP; ++rp) {
-                    ffma2(acc[rp][j], ap[rp][0], d0);
-                    ffma2(acc[rp][j], ap[rp][1], d1);
-                    ffma2(acc[rp][j], ap[rp][2], d2);
-                    ffma2(acc[rp][j], ap[rp][3], d3);
-                }
-            }
-        } else {
-            float2 wd[4][NC];
+        for (int r = 0; r < MB; ++r)
 #pragma unroll
-            for (int j = 0; j < NC; ++j) {
-                const uint2 raw = w_at(j, q);
-                const float w0 = bf16lo(raw.x), w1 = bf16hi(raw.x), w2 = bf16lo(raw.y), w3 = bf16hi(raw.y);
-                wd[0][j] = make_float2(w0, w0);
-                wd[1][j] = make_float2(w1, w1);
-                wd[2][j] = make_float2(w2, w2);
-                wd[3][j] = make_float2(w3, w3);
-            }
+            for (int j = 0; j < NC; ++j) fma_bf16<0>(acc[r][j], ar[r].x, wr[j].x);  // k = 4q
 #pragma unroll
-            for (int rp = 0; rp < RP; ++rp) {
-                const uint2 r0 = a_at(2 * rp, q), r1 = a_at(2 * rp + 1, q);
-                const float2 a0 = make_float2(bf16lo(r0.x), bf16lo(r1.x));
-                const float2 a1 = make_float2(bf16hi(r0.x), bf16hi(r1.x));
-                const float2 a2 = make_float2(bf16lo(r0.y), bf16lo(r1.y));
-                const float2 a3 = make_float2(bf16hi(r0.y), bf16hi(r1.y));
+        for (int r = 0; r < MB; ++r)
 #pragma unroll
-                for (int j = 0; j < NC; ++j) {
-                    ffma2(acc[rp][j], a0, wd[0][j]);
-                    ffma2(acc[rp][j], a1, wd[1][j]);
-                    ffma2(acc[rp][j], a2, wd[2][j]);
-                    ffma2(acc[rp][j], a3, wd[3][j]);
-                }
-            }
-        }
+            for (int j = 0; j < NC; ++j) fma_bf16<1>(acc[r][j], ar[r].x, wr[j].x);  // 4q + 1
+#pragma unroll
+        for (int r = 0; r < MB; ++r)
+#pragma unroll
+            for (int j = 0; j < NC; ++j) fma_bf16<0>(acc[r][j], ar[r].y, wr[j].y);  // 4q + 2
+#pragma unroll
+        for (int r = 0; r < MB; ++r)
+#pragma unroll
+            for (int j = 0; j < NC; ++j) fma_bf16<1>(acc[r][j], ar[r].y, wr[j].y);  // 4q + 3
     }
     // Every accumulator is final before the slot is released: the empty
     // volatile asm consumes them all, and volatile asm keeps its order, so no
     // load of the slot (nor the FMAs that use it) can sink below the release.
 #pragma unroll
-    for (int rp = 0; rp < RP; ++rp)
+    for (int r = 0; r < MB; ++r)
 #pragma unroll
-        for (int j = 0; j < NC; ++j) asm volatile("" ::"f"(acc[rp][j].x), "f"(acc[rp][j].y));
+        for (int j = 0; j < NC; ++j) asm volatile("" ::"f"(acc[r][j]));
     // This warp no longer reads the slot.
     __syncwarp();
     if (lane == 0 && !warm) mbar_arrive(smem_u32(&sm.empty[slot]));
@@ -388,12 +367,9 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     constexpr int V = MB * NC;
     float v[V];
 #pragma unroll
-    for (int rp = 0; rp < RP; ++rp)
+    for (int r = 0; r < MB; ++r)
 #pragma unroll
-        for (int j = 0; j < NC; ++j) {
-            v[(2 * rp) * NC + j] = acc[rp][j].x;
-            v[(2 * rp + 1) * NC + j] = acc[rp][j].y;
-        }
+        for (int j = 0; j < NC; ++j) v[r * NC + j] = acc[r][j];
     int base = 0;
     ReduceScatter<V, 16>::run(v, lane, base);
     constexpr int PL = Scatter<V>::kPerLane;
@@ -684,6 +660,9 @@ inline int col_group_rt(int MB, int k) { return (MB <= 8 && k <= MR_GEMV_CG8_MAX
 template <bool FUSED>
 KernelFn kernel_for_mb(int MB, int CG) {
     switch (MB) {
+        case 1:  // the fused router has no one-row bucket (see row_bucket)
+            if constexpr (!FUSED) return CG == 8 ? gemv_kernel<1, 8, false> : gemv_kernel<1, 4, false>;
+            return nullptr;
         case 2: return CG == 8 ? gemv_kernel<2, 8, FUSED> : gemv_kernel<2, 4, FUSED>;
         case 4: return CG == 8 ? gemv_kernel<4, 8, FUSED> : gemv_kernel<4, 4, FUSED>;
         case 8: return CG == 8 ? gemv_kernel<8, 8, FUSED> : gemv_kernel<8, 4, FUSED>;
@@ -695,8 +674,14 @@ KernelFn kernel_for(int MB, int CG, bool fused) {
     return fused ? kernel_for_mb<true>(MB, CG) : kernel_for_mb<false>(MB, CG);
 }
 
-// Rows are processed in pairs, so a single row runs in the 2-row kernel with a zero second row.
-int row_bucket(int m) { return m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16; }
+// Row bucket of a call: the kernel instance for the smallest bucket that
+// holds m rows.  The fused router runs one row in the 2-row kernel: in a
+// sequence of router windows (m = 1, 2, 4, 8, 16) a one-row fused kernel made
+// the sequence slower (1.06 against 1.02 us a row), while the plain GEMV at
+// m = 1 is 8-11% faster with its one-row kernel.
+int row_bucket(int m, bool fused) {
+    return (m == 1 && !fused) ? 1 : m <= 2 ? 2 : m <= 4 ? 4 : m <= 8 ? 8 : 16;
+}
 
 std::mutex g_attr_mutex;
 bool g_attr_done[64] = {};
@@ -705,12 +690,13 @@ cudaError_t ensure_attributes(int device) {
     std::lock_guard<std::mutex> lock(g_attr_mutex);
     if (device >= 0 && device < 64 && g_attr_done[device]) return cudaSuccess;
     const int optin = mr_host::max_smem_optin();
-    const int mbs[] = {2, 4, 8, 16};
+    const int mbs[] = {1, 2, 4, 8, 16};
     for (int mb : mbs)
         for (int cg = 4; cg <= 8; cg += 4)
             for (int fused = 0; fused < 2; ++fused) {
-                cudaError_t e = cudaFuncSetAttribute(kernel_for(mb, cg, fused != 0),
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+                const KernelFn fn = kernel_for(mb, cg, fused != 0);
+                if (!fn) continue;
+                cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
                 if (e != cudaSuccess) return e;
         }
     if (device >= 0 && device < 64) g_attr_done[device] = true;
@@ -762,7 +748,7 @@ mr_status make_plan(int m, int n, int k, uint32_t flags, int sms, int optin, Pla
     if (m < 1 || n < 1 || k < 8 || sms < 1 || optin < 1) return MR_ERR_INVALID_ARG;
     if (k % 8 != 0) return MR_ERR_MISALIGNED;
     if (m > kMaxRows) return MR_ERR_UNSUPPORTED;
-    pl.MB = row_bucket(m);
+    pl.MB = row_bucket(m, fused);
     pl.CG = col_group_rt(pl.MB, k);
     pl.KW = k_warps(k);
     pl.G = std::min(sms, n);
@@ -907,6 +893,7 @@ mr_status enqueue(const Params &p, const Plan &pl, uint32_t flags, bool fused, v
     cfg.gridDim = dim3((unsigned)p.G);
     // One warm warp beside the GEMV warps when the SM has room for it.
     const KernelFn fn = kernel_for(pl.MB, pl.CG, fused);
+    if (!fn) return MR_ERR_UNSUPPORTED;
     const int warps = p.KW * p.CWG + (warm_warp_fits(fn, p.KW * p.CWG, pl.smem) ? 1 : 0);
     cfg.blockDim = dim3((unsigned)(warps * 32));
     cfg.dynamicSmemBytes = pl.smem;
