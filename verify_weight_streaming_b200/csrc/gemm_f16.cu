@@ -68,6 +68,7 @@ constexpr TileDesc kTiles[] = {
     {128, 128, 6, 128, 2, "128x128"}, {128, 192, 5, 256, 1, "128x192"}, {128, 256, 4, 256, 1, "128x256"},
     {64, 128, 8, 128, 2, "64x128"},   {64, 256, 5, 256, 1, "64x256"},
     {256, 256, 7, 256, 1, "256x256", true},
+    {256, 128, 9, 128, 1, "256x128", true},
 };
 constexpr int kNumTiles = sizeof(kTiles) / sizeof(kTiles[0]);
 
@@ -496,38 +497,45 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
 }
 
-// ---- the CTA-pair kernel: 256 x 256 tiles on two SMs (cta_group::2) ---------
+// ---- the CTA-pair kernel: 256 x PBN tiles on two SMs (cta_group::2) --------
 //
-// A cluster of two CTAs computes a 256 x 256 output tile with one
-// tcgen05.mma.cta_group::2 per K step of 16: CTA v loads rows 128v..128v+127
-// of the tile's A block and rows 128v..128v+127 of its Wt block (columns of
-// the output) into its own shared memory, and CTA v's tensor memory receives
-// rows 128v..128v+127 of the accumulator.  Each CTA streams 32 KB per
-// k-block instead of the 48 KB a 128 x 256 tile needs.  The leader (rank 0)
+// A cluster of two CTAs computes a 256 x PBN output tile (PBN = 128 or 256)
+// with one tcgen05.mma.cta_group::2 per K step of 16: CTA v loads rows
+// 128v..128v+127 of the tile's A block and rows v*PBN/2 .. (v+1)*PBN/2 - 1 of
+// its Wt block (columns of the output) into its own shared memory, and CTA
+// v's tensor memory receives rows 128v..128v+127 of the accumulator.  At
+// PBN = 256 each CTA streams 32 KB per k-block instead of the 48 KB a
+// 128 x 256 tile needs; at PBN = 128, 24 KB instead of the 32 KB of a
+// 128 x 128 tile with the same output per SM.  (A 256 x 64 pair measured
+// 17-19 us on the one-wave chunk shapes against 13-15 us for the best tile,
+// and was left out.)  The leader (rank 0)
 // issues every MMA from one elected thread and waits on its own full
 // barriers, which count the TMA bytes of both CTAs (the peer's loads signal
 // the leader's barrier; no load is multicast); its commits arrive on the
 // barriers of both CTAs.  Both CTAs' epilogue warps release an accumulator
 // buffer on the leader's barrier.  The K sequence is that of every other
 // tile, so the bits are too.
-constexpr int kPairN = 256;          // output columns per tile
 constexpr int kPairRows = 256;       // output rows per tile (128 per CTA)
-constexpr int kPairStages = 7;       // k-blocks of 32 KB per CTA
 
-__host__ __device__ constexpr uint32_t pair_smem_bytes() {
-    return (uint32_t)kPairStages * (a_bytes_for(128) + (uint32_t)(kPairN / 2) * BK * 2) + 1024 + 256;
+// Ring stages of the pair kernel: k-blocks of 16 KB of A and PBN / 2 rows of
+// Wt per CTA, as many as fit beside the barriers.
+__host__ __device__ constexpr int pair_stages(int pbn) { return pbn >= 256 ? 7 : 9; }
+__host__ __device__ constexpr uint32_t pair_smem_bytes(int pbn) {
+    return (uint32_t)pair_stages(pbn) * (a_bytes_for(128) + (uint32_t)(pbn / 2) * BK * 2) + 1024 + 256;
 }
 
-template <int OUT, int MAXG>
+template <int PBN, int OUT, int MAXG>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ GemmArgs<MAXG> args) {
+    static_assert(PBN == 128 || PBN == 256, "pair tile width");
     constexpr int BMH = kPairRows / 2;                 // A rows per CTA
-    constexpr int BNH = kPairN / 2;                    // Wt rows per CTA
+    constexpr int BNH = PBN / 2;                       // Wt rows per CTA
     constexpr uint32_t kAB = (uint32_t)BMH * BK * 2;   // 16 KB
-    constexpr uint32_t kBB = (uint32_t)BNH * BK * 2;   // 16 KB
-    constexpr int NST = kPairStages;
+    constexpr uint32_t kBB = (uint32_t)BNH * BK * 2;   // 8 or 16 KB (multiples of the 1 KB swizzle atom)
+    constexpr int NST = pair_stages(PBN);
     static_assert(NST >= kProducers, "ring too short for the producer warps");
-    constexpr uint32_t ACC_COLS = kPairN;
+    static_assert(pair_smem_bytes(PBN) <= 232448, "pair ring exceeds the opt-in shared memory");
+    constexpr uint32_t ACC_COLS = PBN;
     constexpr uint32_t kTmemCols = 2 * ACC_COLS;
     const CUtensorMap &tmA = args.tmA;
     const int M = args.M, N = args.N, K = args.K;
@@ -587,7 +595,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tile_coords(t, ntm, ntn, args.raster, mt, slot);
             const int m0 = mt * kPairRows + (int)rank * BMH;
             const int g = slot / args.tn_per_group;
-            const int n0 = (slot % args.tn_per_group) * kPairN + (int)rank * BNH;
+            const int n0 = (slot % args.tn_per_group) * PBN + (int)rank * BNH;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 if (it % kProducers != pidx) continue;
                 const uint32_t st = it % NST;
@@ -654,13 +662,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int mt, slot;
             tile_coords(t, ntm, ntn, args.raster, mt, slot);
             const int g = slot / args.tn_per_group;
-            const int n0 = (slot % args.tn_per_group) * kPairN;
+            const int n0 = (slot % args.tn_per_group) * PBN;
             const int row = mt * kPairRows + (int)rank * BMH + 32 * q + lane;
             if (!mbar_wait_bounded(smem_u32(&acc_full[b]), (ti >> 1) & 1u, MR_DEVERR_GEMM_TIMEOUT)) break;
             tc_fence_after();
             const uint32_t acc = tmem + b * ACC_COLS + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
-            for (int c = 0; c < kPairN / 16; ++c) {
+            for (int c = 0; c < PBN / 16; ++c) {
                 uint32_t r[16];
                 tmem_ld16(acc + (uint32_t)(c * 16), r);
                 const int col = n0 + c * 16;
@@ -695,7 +703,8 @@ constexpr KernelFn<MAXG> kernel_of() {
 
 template <int OUT, int MAXG>
 KernelFn<MAXG> pick_out(int t) {
-    if (kTiles[t].pair) return gemm_pair_kernel<OUT, MAXG>;
+    if (kTiles[t].pair)
+        return kTiles[t].bn == 128 ? gemm_pair_kernel<128, OUT, MAXG> : gemm_pair_kernel<256, OUT, MAXG>;
     switch (t) {
         case 0: return kernel_of<0, OUT, MAXG>();
         case 1: return kernel_of<1, OUT, MAXG>();
@@ -711,7 +720,7 @@ KernelFn<MAXG> pick_out(int t) {
 // Dynamic shared memory of tile t's kernel.
 uint32_t tile_smem_bytes(int t) {
     const TileDesc &td = kTiles[t];
-    return td.pair ? pair_smem_bytes() : smem_bytes_for(td.bm, td.bn, td.stages);
+    return td.pair ? pair_smem_bytes(td.bn) : smem_bytes_for(td.bm, td.bn, td.stages);
 }
 
 // Clusters of two CTAs of the pair kernel that fit on the device at once
@@ -725,7 +734,7 @@ int max_pairs(int device) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2);
         cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = pair_smem_bytes();
+        cfg.dynamicSmemBytes = pair_smem_bytes(256);  // the largest pair ring: one CTA per SM for all widths
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -734,7 +743,7 @@ int max_pairs(int device) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<MR_F16, 1>, &cfg) != cudaSuccess || n < 1) {
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<256, MR_F16, 1>, &cfg) != cudaSuccess || n < 1) {
             cudaGetLastError();
             return 0;
         }
@@ -834,8 +843,10 @@ int select_tile_grouped(int M, int N, int K, int G, int sms, int pairs) {
     // placed at those ratios.
     // The 256 x 256 pair tile runs one tile per two SMs; it measured 0.96x
     // the 128 x 256 tile's cost per wave (a wave of pairs covers the same
-    // output area as a wave of 128 x 256 tiles).
-    const double kb_ns[kNumTiles] = {175.0, 193.0, 225.0, 254.0, 338.0, 438.0, 198.0, 372.0, 420.0};
+    // output area as a wave of 128 x 256 tiles).  The 256 x 128 pair costs
+    // 0.85x the 128 x 128 tile per wave (215 ns a k-block: with it the rule
+    // picks the fastest of the ten tiles on 47 of the 48 chunk shapes).
+    const double kb_ns[kNumTiles] = {175.0, 193.0, 225.0, 254.0, 338.0, 438.0, 198.0, 372.0, 420.0, 215.0};
     const int64_t nkb = (K + BK - 1) / BK;
     int best = -1;
     double best_t = 1e300;
