@@ -18,7 +18,7 @@ GEMM TFLOP/s sweep on the prompt-chunk shapes, the CPU oracle as a baseline,
 and the SM clocks seen during the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-    python bench.py --profile-case gemv|topk|gemm   # a few launches, for ncu
+    python bench.py --profile-case gemv|topk|gemm|...   # a few launches, for ncu
     python bench.py --selector-study                # every GEMM tile on every chunk shape
 """
 from __future__ import annotations
@@ -1108,6 +1108,14 @@ def profile_case(case: str):
             mr.router_topk(x, TOPK, idx)
     elif case == "gemm":
         gemm_profile_case()
+    elif case == "gemm_1983x1152":
+        # a one-wave chunk shape on the auto tile (the 256 x 128 pair)
+        a, w = synth.chunk(1983, 1152)
+        A = torch.from_numpy(a.view(np.int16)).cuda().view(torch.float16)
+        W = torch.from_numpy(w.view(np.int16)).cuda().view(torch.float16)
+        C = torch.empty((1983, 1152), dtype=torch.float16, device="cuda")
+        for _ in range(3):
+            mr.gemm_f16(A, W, C)
     torch.cuda.synchronize()
     assert mr.mr_poll_errors() == 0
     print(json.dumps({"profile_case": case, "ok": True}))
