@@ -280,9 +280,9 @@ mr_status cast_f32_bf16(const float *X, int64_t ldx, void *Y, int64_t ldy, int32
  * tile_id : -1 selects with gemm_f16_select_tile; 0 .. gemm_f16_num_tiles()-1
  *      forces a tile.  The family: 128 x {32, 64, 96, 128, 192, 256} (MMA
  *      M = 128), 64 x {128, 256} (MMA M = 64, half the padding of a tail
- *      tile), and 256 x 256 and 256 x 128 computed by a cluster of two CTAs
- *      on two SMs (tcgen05.mma.cta_group::2, M = 256), in that order (ids 0
- *      to 9).  Every tile gives the same bits
+ *      tile), 256 x 256 and 256 x 128 computed by a cluster of two CTAs on
+ *      two SMs (tcgen05.mma.cta_group::2, M = 256), then 64 x {32, 64}, in
+ *      that order (ids 0 to 11).  Every tile gives the same bits
  *      (fixed K order, K steps of 16, no split-K).
  * M, N >= 1; K >= 8, K % 8 == 0; lda, ldw, ldc % 8 == 0; A, Wt, C 16-byte aligned.
  */

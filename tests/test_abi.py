@@ -91,7 +91,7 @@ def gemm(A=A16, lda=64, W=A16, ldw=64, C=A16, ldc=32, M=4, N=32, K=64, ind=mr.MR
     (dict(N=0), mr.MR_ERR_INVALID_ARG), (dict(K=0), mr.MR_ERR_INVALID_ARG),
     (dict(lda=56), mr.MR_ERR_INVALID_ARG), (dict(ldc=24), mr.MR_ERR_INVALID_ARG),
     (dict(ind=mr.MR_F32), mr.MR_ERR_INVALID_ARG), (dict(outd=7), mr.MR_ERR_INVALID_ARG),
-    (dict(tile=10), mr.MR_ERR_INVALID_ARG), (dict(tile=-2), mr.MR_ERR_INVALID_ARG),
+    (dict(tile=12), mr.MR_ERR_INVALID_ARG), (dict(tile=-2), mr.MR_ERR_INVALID_ARG),
     (dict(K=60, lda=64, ldw=64), mr.MR_ERR_MISALIGNED), (dict(ldc=36), mr.MR_ERR_MISALIGNED),
     (dict(C=P(264)), mr.MR_ERR_MISALIGNED), (dict(A=BAD), mr.MR_ERR_MISALIGNED),
 ])
@@ -101,10 +101,10 @@ def test_gemm_validation(kw, code):
 
 def test_gemm_tiles_and_selector_on_host():
     n = mr.gemm_f16_num_tiles()
-    assert n == 10
+    assert n == 12
     names = [mr.gemm_f16_tile_name(t) for t in range(n)]
     assert names == ["128x32", "128x64", "128x96", "128x128", "128x192", "128x256", "64x128", "64x256",
-                     "256x256", "256x128"]
+                     "256x256", "256x128", "64x32", "64x64"]
     assert mr.gemm_f16_tile_name(n) is None and mr.gemm_f16_tile_name(-1) is None
     assert mr.gemm_f16_select_tile(0, 96, 2560) == -1
     for M in (1, 150, 306, 1983, 2048):
@@ -124,12 +124,12 @@ def test_selector_tail_rule_and_measured_choices():
         for rt in (3, 10, 21, 32):
             picks = {mr.gemm_f16_select_tile(M, N, 2560) for M in (64 * (rt - 1) + 1, 64 * rt - 17, 64 * rt)}
             assert len(picks) == 1, (N, rt, picks)
-    measured_best = {(306, 512): "128x32", (306, 640): "128x32", (448, 640): "128x32", (700, 640): "128x32",
-                     (150, 1152): "128x32", (306, 1152): "128x32", (448, 1152): "128x32",
+    measured_best = {(1983, 1152): "256x128", (150, 1664): "64x64", (192, 1664): "64x64", (306, 1664): "64x64",
                      (700, 1664): "64x128", (1300, 1664): "128x128", (1983, 1664): "128x192",
                      (2048, 1664): "128x192", (448, 4096): "256x128", (700, 4096): "128x192",
                      (1983, 4096): "256x256", (2048, 4096): "256x256", (306, 6144): "128x128",
-                     (448, 6144): "128x192", (1983, 6144): "256x256", (2048, 6144): "256x256"}
+                     (448, 6144): "128x192", (1300, 6144): "256x256", (1983, 6144): "256x256",
+                     (2048, 6144): "256x256"}
     for (M, N), name in measured_best.items():
         assert names[mr.gemm_f16_select_tile(M, N, 2560)] == name, (M, N)
 

@@ -69,9 +69,12 @@ constexpr TileDesc kTiles[] = {
     {64, 128, 8, 128, 2, "64x128"},   {64, 256, 5, 256, 1, "64x256"},
     {256, 256, 7, 256, 1, "256x256", true},
     {256, 128, 9, 128, 1, "256x128", true},
+    {64, 32, 12, 32, 2, "64x32"},     {64, 64, 12, 64, 2, "64x64"},
 };
 constexpr int kNumTiles = sizeof(kTiles) / sizeof(kTiles[0]);
 
+// The barriers (2 per k-block slot, 4 for the accumulators) and the tensor
+// memory address take the 256 bytes after the ring: at most 13 slots.
 __host__ __device__ constexpr uint32_t smem_bytes_for(int bm, int bn, int stages) {
     return (uint32_t)stages * (a_bytes_for(bm) + (uint32_t)bn * BK * 2) + 1024 /*align*/ + 256 /*barriers*/;
 }
@@ -332,6 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     // more than one phase ahead of the barrier.
     constexpr int NST = STAGES / KPB;
     static_assert(NST >= kProducers, "ring too short for the producer warps");
+    static_assert((2 * STAGES + 4) * 8 + 4 <= 256, "barriers exceed their 256 bytes");
+    static_assert(smem_bytes_for(BM, BN, STAGES) <= 232448, "ring exceeds the opt-in shared memory");
     uint64_t *full = bars;                    // [NST] TMA -> MMA
     uint64_t *empty = bars + STAGES;          // [NST] MMA -> TMA
     uint64_t *acc_full = bars + 2 * STAGES;   // [2] MMA -> epilogue
@@ -535,6 +540,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     constexpr int NST = pair_stages(PBN);
     static_assert(NST >= kProducers, "ring too short for the producer warps");
     static_assert(pair_smem_bytes(PBN) <= 232448, "pair ring exceeds the opt-in shared memory");
+    static_assert((2 * NST + 4) * 8 + 4 <= 256, "barriers exceed their 256 bytes");
     constexpr uint32_t ACC_COLS = PBN;
     constexpr uint32_t kTmemCols = 2 * ACC_COLS;
     const CUtensorMap &tmA = args.tmA;
@@ -713,6 +719,8 @@ KernelFn<MAXG> pick_out(int t) {
         case 4: return kernel_of<4, OUT, MAXG>();
         case 5: return kernel_of<5, OUT, MAXG>();
         case 6: return kernel_of<6, OUT, MAXG>();
+        case 10: return kernel_of<10, OUT, MAXG>();
+        case 11: return kernel_of<11, OUT, MAXG>();
         default: return kernel_of<7, OUT, MAXG>();
     }
 }
@@ -844,9 +852,11 @@ int select_tile_grouped(int M, int N, int K, int G, int sms, int pairs) {
     // The 256 x 256 pair tile runs one tile per two SMs; it measured 0.96x
     // the 128 x 256 tile's cost per wave (a wave of pairs covers the same
     // output area as a wave of 128 x 256 tiles).  The 256 x 128 pair costs
-    // 0.85x the 128 x 128 tile per wave (215 ns a k-block: with it the rule
-    // picks the fastest of the ten tiles on 47 of the 48 chunk shapes).
-    const double kb_ns[kNumTiles] = {175.0, 193.0, 225.0, 254.0, 338.0, 438.0, 198.0, 372.0, 420.0, 215.0};
+    // 0.85x the 128 x 128 tile per wave (215 ns a k-block), and the 64 x 32
+    // and 64 x 64 tiles 0.91x and 0.93x the 128 x 32 tile (one-wave shapes):
+    // with these the rule picks the fastest of the twelve tiles on 47 of the
+    // 48 chunk shapes.
+    const double kb_ns[kNumTiles] = {175.0, 193.0, 225.0, 254.0, 338.0, 438.0, 198.0, 372.0, 420.0, 215.0, 159.0, 163.0};
     const int64_t nkb = (K + BK - 1) / BK;
     int best = -1;
     double best_t = 1e300;
@@ -854,6 +864,11 @@ int select_tile_grouped(int M, int N, int K, int G, int sms, int pairs) {
         const int bn = kTiles[t].bn;
         const bool pair = kTiles[t].pair;
         if (pair && pairs < 1) continue;
+        // A pair tile holds one group: with several groups narrower than the
+        // tile, its spare columns are work the packed one-CTA tiles avoid
+        // (the 36 projections of N = 96 at M = 512: 13.1 us on 256 x 128
+        // against 12.4 us on 128 x 96).
+        if (pair && G > 1 && N < bn) continue;
         const int P = pack_factor(bn, N, G, pair);
         const int bm = kTiles[t].bm;
         const int64_t tiles = (int64_t)((M + bm - 1) / bm) * n_slots(bn, N, G, P);
