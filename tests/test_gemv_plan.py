@@ -67,3 +67,12 @@ def test_plan_rejects_like_the_entry_point():
     with pytest.raises(mr.MrError) as e:
         mr.mrgemv_bf16_plan(16, 512, 1 << 16, 0, SMS, OPTIN)
     assert e.value.status == mr.MR_ERR_UNSUPPORTED
+
+
+def test_row_buckets():
+    """One row runs in its own kernel; then 2, 4, 8 and 16 rows."""
+    want = {1: 1, 2: 2, 3: 4, 4: 4, 5: 8, 8: 8, 9: 16, 16: 16}
+    for m, mb in want.items():
+        for n, k in ((512, 2560), (4864, 896), (6144, 2560)):
+            assert mr.mrgemv_bf16_plan(m, n, k, mr.MR_GEMV_PDL, SMS, OPTIN)["row_bucket"] == mb, (m, n, k)
+
