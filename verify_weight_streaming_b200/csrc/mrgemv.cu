@@ -62,12 +62,17 @@ namespace gemv {
 // of fewer warps then leaves room on its SM for the next launch's CTA), and
 // the unroll of the k loop: two steps, except for 8-column groups of 4 or more
 // rows and for 16 rows, whose accumulators leave few registers for a second
-// step (measured: one step is faster there, two elsewhere).  None of this
-// changes an output's arithmetic: a lane's chain and the reduction order are
-// fixed by k.
+// step (measured: one step is faster there, two elsewhere), and except in the
+// fused router's kernels, whose code is fetched cold in each window of a
+// sequence of window sizes: one step, half the loop's code, made the window
+// sequence 1-3% faster (same box) though a repeated m = 1 window is 0.1 us
+// slower.  None of this changes an output's arithmetic: a lane's chain and
+// the reduction order are fixed by k.
 constexpr int kWarpsMax = 16;
 __host__ __device__ constexpr int warps_max(int, int) { return kWarpsMax; }
-__host__ __device__ constexpr int q_unroll(int MB, int CG) { return ((CG >= 8 && MB >= 4) || MB >= 16) ? 1 : 2; }
+__host__ __device__ constexpr int q_unroll(int MB, int CG, bool fused = false) {
+    return (fused || (CG >= 8 && MB >= 4) || MB >= 16) ? 1 : 2;
+}
 
 constexpr int kMaxRows = 16;
 // Fused router: each logit is also stored as one 64-bit word, the flag
@@ -329,7 +334,7 @@ __device__ __forceinline__ bool do_group(const Params &p, const Smem &sm, int g,
     // mixed-precision FMA, so consecutive FMAs are independent of each other.
     auto a_at = [&](int r, int qq) { return lds64(a_s + (uint32_t)r * row_b + 8u * (uint32_t)qq); };
     auto w_at = [&](int j, int qq) { return lds64(w_s + (uint32_t)j * row_b + 8u * (uint32_t)qq); };
-#pragma unroll (q_unroll(MB, CGMAX))
+#pragma unroll (q_unroll(MB, CGMAX, FUSED))
     for (int q = q_begin + lane; q < q_end; q += 32) {
         uint2 wr[NC], ar[MB];
 #pragma unroll
@@ -506,7 +511,7 @@ __global__ void __launch_bounds__(kWarpsMax * 32, 1) gemv_kernel(const Params p)
     const int q_total = k / 4;
     const int q_begin = (int)(((int64_t)slice * q_total) / p.KW);
     const int q_end = (int)(((int64_t)(slice + 1) * q_total) / p.KW);
-    constexpr int kQStep = 32 * q_unroll(MB, CG);  // one unrolled step of the k loop
+    constexpr int kQStep = 32 * q_unroll(MB, CG, FUSED);  // one unrolled step of the k loop
 
     // The GEMV warps are 0 .. KW * CWG - 1.  A launch with fewer than 16 of
     // them has one more warp, which runs the code below once at kernel start
